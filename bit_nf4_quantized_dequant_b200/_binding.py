@@ -1,3 +1,217 @@
-"""ctypes binding of libqlora (filled in with the C ABI)."""
+"""ctypes binding of libqlora: argument marshalling only.
 
-__all__ = []
+Every call maps one-to-one onto a C entry point of ``include/qlora.h``; torch
+supplies device memory (output tensors are allocated with torch when the
+caller passes none) and the current CUDA stream. No step of the computation
+runs here. If the shared library is missing or cannot be loaded, every call
+raises ``QloraUnavailable``; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "QloraError", "QloraUnavailable", "NF4Matrix", "library", "library_path", "SYMBOLS",
+    "nf4_sizes", "nf4_codebook", "nf4_quantize", "nf4_dequantize",
+    "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libqlora.so")
+
+STATUS = {
+    0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED_SHAPE",
+    3: "QLORA_ERR_MISALIGNED", 4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_NONFINITE",
+    6: "QLORA_ERR_TIMEOUT", 7: "QLORA_ERR_CUDA",
+}
+
+# every symbol include/qlora.h declares
+SYMBOLS = [
+    "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_nf4_quantize", "qlora_nf4_dequantize",
+    "qlora_linear_workspace", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
+]
+
+
+class QloraUnavailable(RuntimeError):
+    """libqlora.so is missing or failed to load."""
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call} returned {STATUS.get(status, status)}")
+
+
+class _NF4(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scale8", ctypes.c_void_p), ("scale2", ctypes.c_void_p)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def library():
+    """The loaded shared library (loaded once)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise QloraUnavailable(f"{library_path} not built (run bit_nf4_quantized_dequant_b200._build)")
+    try:
+        lib = ctypes.CDLL(library_path)
+    except OSError as e:  # pragma: no cover - depends on the machine
+        raise QloraUnavailable(f"cannot load {library_path}: {e}") from e
+    st = ctypes.c_int
+    lib.qlora_nf4_sizes.argtypes = [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]
+    lib.qlora_nf4_sizes.restype = st
+    lib.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
+    lib.qlora_nf4_codebook.restype = st
+    lib.qlora_nf4_quantize.argtypes = [_P, ctypes.POINTER(_NF4), _P, _P]
+    lib.qlora_nf4_quantize.restype = st
+    lib.qlora_nf4_dequantize.argtypes = [ctypes.POINTER(_NF4), _P, _P]
+    lib.qlora_nf4_dequantize.restype = st
+    lib.qlora_linear_workspace.argtypes = [_I64, _I64, _I64, ctypes.c_int32, ctypes.POINTER(_SZ)]
+    lib.qlora_linear_workspace.restype = st
+    lib.qlora_linear_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, _P, ctypes.c_int32, ctypes.c_float,
+                                     _P, _P, _P, _SZ, _P, _P]
+    lib.qlora_linear_fwd.restype = st
+    lib.qlora_linear_bwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, _P, ctypes.c_int32, ctypes.c_float,
+                                     _P, _P, _P, _P, _P, _P, _SZ, _P, _P]
+    lib.qlora_linear_bwd.restype = st
+    lib.qlora_status_string.argtypes = [ctypes.c_int]
+    lib.qlora_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int, call: str):
+    if status != 0:
+        raise QloraError(status, call)
+
+
+def status_string(status: int) -> str:
+    return library().qlora_status_string(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def nf4_sizes(rows: int, cols: int):
+    """(code bytes, scale8 bytes, scale2 bytes) of a [rows, cols] NF4 matrix."""
+    a, b, c = _SZ(), _SZ(), _SZ()
+    _check(library().qlora_nf4_sizes(rows, cols, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "qlora_nf4_sizes")
+    return a.value, b.value, c.value
+
+
+def nf4_codebook():
+    import numpy as np
+    out = (ctypes.c_float * 16)()
+    _check(library().qlora_nf4_codebook(out), "qlora_nf4_codebook")
+    return np.frombuffer(bytes(out), dtype=np.float32).copy()
+
+
+@dataclass
+class NF4Matrix:
+    """Device buffers of one NF4 matrix (torch uint8/uint8/float32 tensors)."""
+    rows: int
+    cols: int
+    codes: object
+    scale8: object
+    scale2: object
+
+    def c_struct(self) -> _NF4:
+        return _NF4(self.rows, self.cols, self.codes.data_ptr(), self.scale8.data_ptr(), self.scale2.data_ptr())
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, device="cuda"):
+        import torch
+        cb, sb, s2b = nf4_sizes(rows, cols)
+        return cls(rows, cols, torch.empty(cb, dtype=torch.uint8, device=device),
+                   torch.empty(sb, dtype=torch.uint8, device=device),
+                   torch.empty(s2b // 4, dtype=torch.float32, device=device))
+
+
+def nf4_quantize(W, out: NF4Matrix | None = None, status=None, stream=None) -> NF4Matrix:
+    """Quantise a contiguous float32 CUDA tensor W[N, K] (K % 64 == 0)."""
+    rows, cols = W.shape
+    q = out if out is not None else NF4Matrix.empty(rows, cols, W.device)
+    s = q.c_struct()
+    _check(library().qlora_nf4_quantize(_ptr(W), ctypes.byref(s), _ptr(status), _stream(stream)),
+           "qlora_nf4_quantize")
+    return q
+
+
+def nf4_dequantize(q: NF4Matrix, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.codes.device)
+    s = q.c_struct()
+    _check(library().qlora_nf4_dequantize(ctypes.byref(s), _ptr(out), _stream(stream)), "qlora_nf4_dequantize")
+    return out
+
+
+def linear_workspace(M: int, N: int, K: int, r: int) -> int:
+    b = _SZ()
+    _check(library().qlora_linear_workspace(M, N, K, r, ctypes.byref(b)), "qlora_linear_workspace")
+    return b.value
+
+
+def _ws(ws, M, N, K, r, device):
+    import torch
+    need = linear_workspace(M, N, K, r)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def linear_fwd(q: NF4Matrix, X, A, B, s: float, Y=None, sU=None, ws=None, status=None, stream=None,
+               want_sU: bool = True):
+    """Y = X W'^T + s (X A^T) B^T. Returns (Y, sU) with sU = bf16(s X A^T) (or None)."""
+    import torch
+    M, K = X.shape
+    r = A.shape[0]
+    N = q.rows
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if sU is None and want_sU:
+        sU = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    ws = _ws(ws, M, N, K, r, X.device)
+    st = q.c_struct()
+    _check(library().qlora_linear_fwd(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y), _ptr(sU),
+                                      _ptr(ws), ws.numel(), _ptr(status), _stream(stream)), "qlora_linear_fwd")
+    return Y, sU
+
+
+def linear_bwd(q: NF4Matrix, X, A, B, s: float, dY, sU=None, dX=None, dA=None, dB=None, ws=None,
+               status=None, stream=None, want_dX: bool = True):
+    """(dX, dA, dB) of the QLoRA linear; dW is never formed."""
+    import torch
+    M, K = X.shape
+    r = A.shape[0]
+    N = q.rows
+    if dX is None and want_dX:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=X.device)
+    if dA is None:
+        dA = torch.empty((r, K), dtype=torch.float32, device=X.device)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=torch.float32, device=X.device)
+    ws = _ws(ws, M, N, K, r, X.device)
+    st = q.c_struct()
+    _check(library().qlora_linear_bwd(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(dY), _ptr(sU),
+                                      _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _ptr(status),
+                                      _stream(stream)), "qlora_linear_bwd")
+    return dX, dA, dB

@@ -1,0 +1,262 @@
+// The C ABI of libqlora (declared in include/qlora.h): argument validation,
+// workspace layout, tensor-map encoding and kernel launches. Nothing here
+// allocates device memory or synchronises.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "qlora.h"
+#include "qlora_device.cuh"
+#include "qlora_internal.h"
+
+namespace qlora {
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+std::once_flag g_encode_once;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Workspace layout of the linear calls (offsets in bytes, 256-byte aligned):
+//   [sU scratch: M*r bf16][sT: M*r bf16][fp32 partial sums of the skinny products]
+struct WsLayout {
+  size_t su, st, part, part_floats, total;
+};
+
+static WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r) {
+  WsLayout w{};
+  const size_t mr = round_up(static_cast<size_t>(M) * r * 2, 256);
+  w.su = 0;
+  w.st = mr;
+  w.part = 2 * mr;
+  size_t f = lora_rows_ws_floats(M, K, r);
+  f = f > lora_rows_ws_floats(M, N, r) ? f : lora_rows_ws_floats(M, N, r);
+  f = f > lora_cols_ws_floats(M, K, r) ? f : lora_cols_ws_floats(M, K, r);
+  f = f > lora_cols_ws_floats(M, N, r) ? f : lora_cols_ws_floats(M, N, r);
+  w.part_floats = f;
+  w.total = w.part + round_up(f * 4, 256);
+  return w;
+}
+
+static qlora_status_t check_nf4(const qlora_nf4_t *q) {
+  if (!q || !q->codes || !q->scale8 || !q->scale2) return QLORA_ERR_INVALID_ARG;
+  if (q->rows <= 0 || q->cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (q->cols % kBlock) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q->codes)) return QLORA_ERR_MISALIGNED;
+  // scale8 / scale2 are read element-wise by the kernels: natural alignment suffices
+  if (reinterpret_cast<uintptr_t>(q->scale2) & 3u) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+static qlora_status_t check_linear(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                   const uint16_t *B, int32_t r, float s) {
+  qlora_status_t st = check_nf4(W);
+  if (st != QLORA_OK) return st;
+  if (!X || !A || !B || M <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (r < 8 || r > 64 || (r % 8)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (W->rows % 16) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) || W->rows > (int64_t(1) << 31) || W->cols > (int64_t(1) << 31))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+static qlora_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+qlora_status_t qlora_nf4_sizes(int64_t rows, int64_t cols, size_t *codes_bytes, size_t *scale8_bytes,
+                               size_t *scale2_bytes) {
+  if (!codes_bytes || !scale8_bytes || !scale2_bytes || rows <= 0 || cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (cols % kBlock) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(cols);
+  const size_t nb = n / kBlock;
+  *codes_bytes = n / 2;
+  *scale8_bytes = nb;
+  *scale2_bytes = 4 * ((nb + kGroup - 1) / kGroup);
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_nf4_codebook(float *out) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  static const float levels[16] = QLORA_NF4_LEVELS;
+  std::memcpy(out, levels, sizeof(levels));
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_nf4_quantize(const float *W, const qlora_nf4_t *q, int32_t *dev_status,
+                                  qlora_stream_t stream) {
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_quantize(W, q->rows, q->cols, q->codes, q->scale8, q->scale2, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_nf4_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora_stream_t stream) {
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_dequantize(q->codes, q->scale8, q->scale2, q->rows, q->cols, out,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t *bytes) {
+  if (!bytes || M <= 0 || N <= 0 || K <= 0) return QLORA_ERR_INVALID_ARG;
+  if (K % kBlock || N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  *bytes = ws_layout(M, N, K, r).total;
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
+                                void *ws, size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
+  qlora_status_t st = check_linear(W, X, M, A, B, r, s);
+  if (st != QLORA_OK) return st;
+  if (!Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(Y) || (sU_out && !aligned16(sU_out))) return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  const WsLayout L = ws_layout(M, N, K, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(wsb + L.su);
+  float *part = reinterpret_cast<float *>(wsb + L.part);
+
+  cudaError_t e = launch_lora_rows(X, M, K, A, r, /*w_is_rk=*/true, s, sU, part, L.part_floats, cs);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.mode = 0;
+  g.codes = W->codes;
+  g.scale8 = W->scale8;
+  g.scale2 = W->scale2;
+  g.N = N;
+  g.K = K;
+  g.M = M;
+  g.r = r;
+  g.act = X;
+  g.lora_w = B;
+  g.lora_act = sU;
+  g.out = Y;
+  g.dev_status = dev_status;
+  return cuda_status(launch_fused_gemm(g, cs));
+}
+
+qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                const uint16_t *B, int32_t r, float s, const uint16_t *dY,
+                                const uint16_t *sU_in, uint16_t *dX, float *dA, float *dB, void *ws,
+                                size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
+  qlora_status_t st = check_linear(W, X, M, A, B, r, s);
+  if (st != QLORA_OK) return st;
+  if (!dY || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
+      (sU_in && !aligned16(sU_in)))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  const WsLayout L = ws_layout(M, N, K, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  uint16_t *sT = reinterpret_cast<uint16_t *>(wsb + L.st);
+  float *part = reinterpret_cast<float *>(wsb + L.part);
+  const uint16_t *sU = sU_in;
+  cudaError_t e;
+  if (!sU) {
+    uint16_t *su_ws = reinterpret_cast<uint16_t *>(wsb + L.su);
+    e = launch_lora_rows(X, M, K, A, r, true, s, su_ws, part, L.part_floats, cs);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    sU = su_ws;
+  }
+  // sT = bf16(s * dY B)
+  e = launch_lora_rows(dY, M, N, B, r, /*w_is_rk=*/false, s, sT, part, L.part_floats, cs);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dX) {
+    GemmArgs g{};
+    g.mode = 1;
+    g.codes = W->codes;
+    g.scale8 = W->scale8;
+    g.scale2 = W->scale2;
+    g.N = N;
+    g.K = K;
+    g.M = M;
+    g.r = r;
+    g.act = dY;
+    g.lora_w = A;
+    g.lora_act = sT;
+    g.out = dX;
+    g.dev_status = dev_status;
+    e = launch_fused_gemm(g, cs);
+    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  }
+  // dA[j, k] = sum_m sT[m, j] X[m, k];  dB[n, j] = sum_m dY[m, n] sU[m, j]
+  e = launch_lora_cols(X, M, K, sT, r, /*transpose_out=*/true, dA, part, L.part_floats, cs);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  e = launch_lora_cols(dY, M, N, sU, r, /*transpose_out=*/false, dB, part, L.part_floats, cs);
+  return cuda_status(e);
+}
+
+const char *qlora_status_string(qlora_status_t status) {
+  switch (status) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "QLORA_ERR_UNSUPPORTED_SHAPE";
+    case QLORA_ERR_MISALIGNED: return "QLORA_ERR_MISALIGNED";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE";
+    case QLORA_ERR_NONFINITE: return "QLORA_ERR_NONFINITE";
+    case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA";
+  }
+  return "QLORA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

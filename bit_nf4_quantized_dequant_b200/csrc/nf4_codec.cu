@@ -1,0 +1,131 @@
+// NF4 codec kernels: blockwise absmax quantisation with double quantisation of
+// the block constants, and standalone dequantisation to bf16.
+//
+// Format ("QLoRA, in depth", section "The mechanism in brief"; "What is
+// QLoRA ...", section "The three QLoRA ideas"): blocks of 64 consecutive
+// row-major weights, 4-bit codes into the NF4 levels, one 8-bit constant per
+// block, one fp32 second-level scale per group of 256 blocks.
+#include "qlora_device.cuh"
+
+namespace qlora {
+namespace {
+
+// code = number of midpoints between adjacent levels that n lies strictly
+// above: the nearest level, ties to the lower one. The midpoints of two float32
+// levels are exact in float64, and so is the comparison.
+__device__ __forceinline__ uint32_t nearest_level(float n) {
+  constexpr float L[16] = QLORA_NF4_LEVELS;
+  const double x = static_cast<double>(n);
+  uint32_t code = 0;
+#pragma unroll
+  for (int i = 0; i < 15; ++i) {
+    const double mid = 0.5 * (static_cast<double>(L[i]) + static_cast<double>(L[i + 1]));
+    code += (x > mid) ? 1u : 0u;
+  }
+  return code;
+}
+
+// One CTA per group of 256 blocks; warp w handles blocks w, w+8, ...; lane l
+// holds elements 2l and 2l+1 of a block, so the packed byte l of the block is
+// written by lane l.
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restrict__ W, int64_t nb,
+                                                           uint8_t *__restrict__ codes,
+                                                           uint8_t *__restrict__ scale8,
+                                                           float *__restrict__ scale2,
+                                                           int32_t *status) {
+  __shared__ float c1s[kGroup];
+  __shared__ float red[8];
+  const int64_t g = blockIdx.x;
+  const int64_t b0 = g * kGroup;
+  const int nblk = static_cast<int>(nb - b0 < kGroup ? nb - b0 : kGroup);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  bool bad = false;
+  for (int i = warp; i < nblk; i += 8) {
+    const int64_t b = b0 + i;
+    const float2 v = __ldg(reinterpret_cast<const float2 *>(W + b * kBlock) + lane);
+    bad |= !isfinite(v.x) || !isfinite(v.y);
+    float m = fmaxf(fabsf(v.x), fabsf(v.y));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    uint32_t e0 = 7, e1 = 7;
+    if (m > 0.f) {
+      e0 = nearest_level(__fdiv_rn(v.x, m));
+      e1 = nearest_level(__fdiv_rn(v.y, m));
+    }
+    codes[b * (kBlock / 2) + lane] = static_cast<uint8_t>((e0 << 4) | e1);
+    if (lane == 0) c1s[i] = m;
+  }
+  if (bad) set_status(status, 5 /* QLORA_ERR_NONFINITE */);
+  __syncthreads();
+
+  // second level: c2 = max c1 over the group
+  const int t = threadIdx.x;
+  const float c1 = t < nblk ? c1s[t] : 0.f;
+  float m = c1;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  float c2 = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) c2 = fmaxf(c2, red[i]);
+  if (t < nblk) {
+    uint32_t q = 0;
+    if (c2 > 0.f) {
+      // 255 c1 is exact in float64 and the float64 quotient is correctly
+      // rounded; it cannot reach a half-integer unless the exact ratio is one,
+      // so rounding it half-to-even rounds the exact ratio half-to-even.
+      q = static_cast<uint32_t>(rint(__ddiv_rn(255.0 * static_cast<double>(c1), static_cast<double>(c2))));
+    }
+    scale8[b0 + t] = static_cast<uint8_t>(q);
+  }
+  if (t == 0) scale2[g] = __fdiv_rn(c2, 255.0f);
+}
+
+// One thread per half block (32 weights = 16 code bytes -> 64 output bytes).
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
+                                                          const uint8_t *__restrict__ scale8,
+                                                          const float *__restrict__ scale2,
+                                                          int64_t nhalf, uint16_t *__restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= nhalf) return;
+  const int64_t b = i >> 1;
+  const uint4 c = __ldg(reinterpret_cast<const uint4 *>(codes) + i);
+  const float sc = block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
+  const Nf4Table t = make_table(sc);
+  uint4 *dst = reinterpret_cast<uint4 *>(out) + i * 4;
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t o[4];
+    expand8(t, w[q], o);
+    dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s) {
+  const int64_t nb = rows * cols / kBlock;
+  const int64_t ng = (nb + kGroup - 1) / kGroup;
+  if (dev_status) {
+    cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  nf4_quantize_kernel<<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2,
+                                                                dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s) {
+  const int64_t nhalf = rows * cols / 32;
+  const int64_t grid = (nhalf + 255) / 256;
+  nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,52 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qlora {
+
+constexpr int kBlock = 64;    // weights per first-level block
+constexpr int kGroup = 256;   // blocks per second-level group
+
+// Kernel launchers. Each returns the cudaError_t of the launch.
+cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s);
+cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s);
+
+// Fused NF4 GEMM (tcgen05). Mode FWD: Y[M,N] = X[M,K] W'^T + sU[M,r] Bl^T.
+// Mode DX: dX[M,K] = dY[M,N] W' + sT[M,r] Al.
+struct GemmArgs {
+  int mode;                 // 0 = FWD, 1 = DX
+  const uint8_t *codes;
+  const uint8_t *scale8;
+  const float *scale2;
+  int64_t N, K, M;
+  int r;
+  const uint16_t *act;      // X (FWD) or dY (DX), [M, K] or [M, N]
+  const uint16_t *lora_w;   // B [N, r] (FWD) or A [r, K] (DX)
+  const uint16_t *lora_act; // sU or sT [M, r]
+  uint16_t *out;            // Y [M, N] or dX [M, K]
+  int32_t *dev_status;
+};
+cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t s);
+
+// Skinny LoRA products (fp32 accumulation).
+// out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if
+// w_is_rk else W[k*r + j].
+cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint16_t *W, int r,
+                             bool w_is_rk, float s, uint16_t *out, float *ws, size_t ws_floats,
+                             cudaStream_t st);
+// sum over m of Z[m, d] * V[m, j]  ->  out[d*r + j] (transpose_out = false) or
+// out[j*D + d] (transpose_out = true), fp32.
+cudaError_t launch_lora_cols(const uint16_t *Z, int64_t M, int64_t D, const uint16_t *V, int r,
+                             bool transpose_out, float *out, float *ws, size_t ws_floats,
+                             cudaStream_t st);
+size_t lora_rows_ws_floats(int64_t M, int64_t K, int r);
+size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
+
+int device_sm_count();
+
+}  // namespace qlora

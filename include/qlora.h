@@ -1,0 +1,153 @@
+/*
+ * libqlora -- the NF4 QLoRA linear layer on one NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument is either a host pointer (marked "host") or a
+ * device pointer in the current CUDA device's memory (marked "device"). The
+ * library never allocates, frees or synchronises: the caller owns every
+ * buffer, passes scratch space explicitly ("workspace") and reads results
+ * after synchronising the stream itself. Calls are asynchronous on `stream`
+ * (NULL = the legacy default stream). Argument errors are detected on the host
+ * and returned synchronously before anything is launched; errors that only the
+ * GPU can see (non-finite weights, a bounded wait that ran out) are written to
+ * an optional device status word. No C++ exception crosses this boundary.
+ *
+ * Layouts: every matrix is row-major and contiguous; bf16 values are passed as
+ * their 16-bit patterns (uint16_t). Device pointers must be 16-byte aligned.
+ *
+ * Notation: W is the frozen weight [N, K] (N = out features, K = in features),
+ * X the activations [M, K] (M tokens), A the LoRA down matrix [r, K], B the
+ * LoRA up matrix [N, r], s = alpha / r. The layer computes
+ *     Y = X W'^T + s (X A^T) B^T
+ * where W' is the NF4 weight dequantised to bf16 ("QLoRA, in depth", section
+ * "The mechanism in brief": each forward dequantises W to the compute dtype
+ * and adds (alpha / r) B A x; backward gives gradients for A, B and the
+ * activations, never for W).
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,        /* null pointer, bad size, bad scalar */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* a shape the kernels do not cover */
+  QLORA_ERR_MISALIGNED = 3,         /* a device pointer not 16-byte aligned */
+  QLORA_ERR_WORKSPACE = 4,          /* workspace missing or too small */
+  QLORA_ERR_NONFINITE = 5,          /* device status: NaN or inf in a weight */
+  QLORA_ERR_TIMEOUT = 6,            /* device status: a bounded wait ran out */
+  QLORA_ERR_CUDA = 7                /* a CUDA runtime call failed */
+} qlora_status_t;
+
+/* Same type as cudaStream_t; spelled out so this header needs no CUDA header. */
+typedef struct CUstream_st *qlora_stream_t;
+
+/*
+ * An NF4 matrix: a non-owning view of three device buffers.
+ * Format ("QLoRA, in depth", "The mechanism in brief"; "What is QLoRA ...",
+ * "The three QLoRA ideas"): W[rows, cols] is cut into blocks of 64
+ * consecutive row-major elements (cols % 64 == 0, so a block lies inside one
+ * row); each weight is a 4-bit code into the 16-level NF4 codebook; each block
+ * has an 8-bit scale; each group of 256 consecutive blocks has one fp32
+ * second-level scale.
+ *   codes : rows*cols/2 bytes; byte j = (code[2j] << 4) | code[2j+1]
+ *           (the first element of a pair in the high nibble).
+ *   scale8: nb = rows*cols/64 bytes; block b's constant is scale8[b] * scale2[b/256].
+ *   scale2: ng = ceil(nb/256) floats, scale2[g] = RN32(max c1 in group g / 255).
+ * Dequantised weight: w' = bf16_rn(fp32_rn(level[code] * fp32_rn(scale8[b] * scale2[b/256]))).
+ */
+typedef struct {
+  int64_t rows;
+  int64_t cols;
+  uint8_t *codes;
+  uint8_t *scale8;
+  float *scale2;
+} qlora_nf4_t;
+
+/* Byte sizes of the three buffers of a [rows, cols] NF4 matrix (host).
+ * Source: "QLoRA, in depth", "The mechanism in brief" (about 4.127 bits per
+ * weight). Errors: INVALID_ARG on null outputs or rows/cols <= 0,
+ * UNSUPPORTED_SHAPE when cols % 64 != 0. */
+qlora_status_t qlora_nf4_sizes(int64_t rows, int64_t cols, size_t *codes_bytes,
+                               size_t *scale8_bytes, size_t *scale2_bytes);
+
+/* Copies the 16 NF4 levels (float32, ascending, level[0] = -1, level[7] = 0,
+ * level[15] = 1) into out (host, 16 floats). The levels are normal quantiles
+ * ("QLoRA and Fine-Tuning on One Consumer GPU", "NF4 and double
+ * quantisation"). */
+qlora_status_t qlora_nf4_codebook(float *out);
+
+/* Quantise W (device, float32 [q->rows, q->cols]) into q's buffers (device).
+ * Per block: c1 = max|w|; code = nearest level to fp32_rn(w / c1), ties to the
+ * lower level, all-zero block -> code 7; per group: c2 = max c1,
+ * scale8 = round-half-even(255 c1 / c2), scale2 = fp32_rn(c2 / 255).
+ * Source: "QLoRA, in depth", "The mechanism in brief"; "What is QLoRA ...",
+ * "The three QLoRA ideas".
+ * dev_status (device int32, may be NULL): set to 0 by this call, then to
+ * QLORA_ERR_NONFINITE if any weight is NaN or inf (the outputs are then
+ * written but meaningless). Errors returned: INVALID_ARG, UNSUPPORTED_SHAPE,
+ * MISALIGNED, CUDA. */
+qlora_status_t qlora_nf4_quantize(const float *W, const qlora_nf4_t *q,
+                                  int32_t *dev_status, qlora_stream_t stream);
+
+/* Dequantise q (device buffers) into out (device, bf16 [rows, cols]),
+ * bit-exactly by the formula in the qlora_nf4_t comment. Source: "QLoRA, in
+ * depth", "The mechanism in brief" (W is dequantised to the compute dtype,
+ * usually bf16). Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+qlora_status_t qlora_nf4_dequantize(const qlora_nf4_t *q, uint16_t *out,
+                                    qlora_stream_t stream);
+
+/* Workspace bytes that qlora_linear_fwd and qlora_linear_bwd need for M
+ * tokens through an [N, K] layer of rank r (host). The same workspace may be
+ * reused by consecutive calls on one stream; calls that run concurrently need
+ * separate workspaces. Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
+qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r,
+                                      size_t *bytes);
+
+/* Forward of the QLoRA linear: Y = X W'^T + s (X A^T) B^T.
+ * W: NF4 weight [N, K] (struct on the host, buffers on the device).
+ * X [M, K], A [r, K], B [N, r]: device bf16. Y [M, N]: device bf16, written.
+ * sU_out [M, r]: device bf16 or NULL; if given, receives bf16_rn(s X A^T), the
+ *   value the backward can reuse instead of recomputing it.
+ * ws / ws_bytes: device workspace of at least qlora_linear_workspace() bytes.
+ * dev_status: device int32 or NULL; set to QLORA_ERR_TIMEOUT if a bounded wait
+ *   inside a kernel ran out (results are then incomplete). It is not cleared.
+ * Supported: M >= 1, N % 16 == 0, K % 64 == 0, r % 8 == 0 with 8 <= r <= 64,
+ * s finite. fp32 accumulation; W' is dequantised tile by tile in shared memory
+ * and never written to global memory ("QLoRA and Fine-Tuning on One Consumer
+ * GPU", "The idea in one line": each weight tile is dequantised to bf16 only
+ * for the moment it is used in a matmul).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
+qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M,
+                                const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                                uint16_t *Y, uint16_t *sU_out, void *ws, size_t ws_bytes,
+                                int32_t *dev_status, qlora_stream_t stream);
+
+/* Backward of the QLoRA linear with W frozen (no dW is ever formed):
+ *   T  = dY B                  (kept as bf16_rn(s T) in the workspace)
+ *   dX = dY W' + s T A         [M, K] bf16   (skipped when dX == NULL)
+ *   dA = s T^T X               [r, K] fp32   (overwritten)
+ *   dB = s dY^T (X A^T)        [N, r] fp32   (overwritten)
+ * dY [M, N] device bf16. sU (device bf16 [M, r]) is the forward's sU_out; if
+ * NULL it is recomputed from X and A. Other arguments as in qlora_linear_fwd.
+ * Source: "QLoRA, in depth", "The mechanism in brief".
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
+qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M,
+                                const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                                const uint16_t *dY, const uint16_t *sU, uint16_t *dX,
+                                float *dA, float *dB, void *ws, size_t ws_bytes,
+                                int32_t *dev_status, qlora_stream_t stream);
+
+/* A static, human-readable name for a status code (host). */
+const char *qlora_status_string(qlora_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

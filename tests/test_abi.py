@@ -1,0 +1,98 @@
+"""The C-ABI library builds for sm_100a, loads, exports every symbol that
+include/qlora.h declares, and its host-only calls and argument checks behave
+as documented. No kernel is launched here (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import nf4 as onf4, sizes as osizes
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = declared_symbols()
+    assert syms == sorted(lib.SYMBOLS)
+    so = lib.library()
+    for s in syms:
+        assert getattr(so, s) is not None
+
+
+def test_sizes_match_oracle(lib):
+    for rows, cols in [(1024, 1024), (4096, 4096), (11008, 4096), (1, 64 * 257), (48, 192)]:
+        assert lib.nf4_sizes(rows, cols) == osizes.nf4_storage_bytes(rows, cols)
+
+
+def test_codebook_matches_oracle_derivation_bitwise(lib):
+    """The library's hard-coded levels against the oracle's own derivation
+    (bisection quantile function): two independent computations."""
+    assert np.array_equal(lib.nf4_codebook().view(np.uint32), onf4.nf4_levels().view(np.uint32))
+
+
+def test_status_strings(lib):
+    for code, name in lib.STATUS.items():
+        assert lib.status_string(code) == name
+
+
+def _nf4(rows, cols, codes=0x10000, s8=0x20000, s2=0x30000):
+    return lib_struct(rows, cols, codes, s8, s2)
+
+
+def lib_struct(rows, cols, codes, s8, s2):
+    from bit_nf4_quantized_dequant_b200._binding import _NF4
+    return _NF4(rows, cols, codes, s8, s2)
+
+
+def test_argument_errors_are_returned_before_any_launch(lib):
+    so = lib.library()
+    SZ = ctypes.c_size_t
+    a, b, c = SZ(), SZ(), SZ()
+    assert so.qlora_nf4_sizes(16, 100, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 2
+    assert so.qlora_nf4_sizes(0, 64, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 1
+    assert so.qlora_nf4_sizes(16, 64, None, ctypes.byref(b), ctypes.byref(c)) == 1
+    assert so.qlora_nf4_codebook(None) == 1
+    # quantize: null input, bad shape, misaligned pointers
+    q = _nf4(16, 64)
+    assert so.qlora_nf4_quantize(None, ctypes.byref(q), None, None) == 1
+    assert so.qlora_nf4_quantize(ctypes.c_void_p(0x40008), ctypes.byref(q), None, None) == 3
+    q_bad = _nf4(16, 100)
+    assert so.qlora_nf4_quantize(ctypes.c_void_p(0x40000), ctypes.byref(q_bad), None, None) == 2
+    q_mis = _nf4(16, 64, codes=0x10004)
+    assert so.qlora_nf4_dequantize(ctypes.byref(q_mis), ctypes.c_void_p(0x40000), None) == 3
+    assert so.qlora_nf4_dequantize(ctypes.byref(q), None, None) == 1
+    # linear: unsupported rank, shape, null operands, missing workspace
+    P = ctypes.c_void_p
+    X, A, B, Y = P(0x50000), P(0x60000), P(0x70000), P(0x80000)
+    q = _nf4(32, 64)
+    fwd = so.qlora_linear_fwd
+    assert fwd(ctypes.byref(q), X, 8, A, B, 12, 2.0, Y, None, None, 0, None, None) == 2
+    assert fwd(ctypes.byref(q), X, 8, A, B, 72, 2.0, Y, None, None, 0, None, None) == 2
+    assert fwd(ctypes.byref(q), None, 8, A, B, 16, 2.0, Y, None, None, 0, None, None) == 1
+    assert fwd(ctypes.byref(q), X, 0, A, B, 16, 2.0, Y, None, None, 0, None, None) == 1
+    assert fwd(ctypes.byref(q), X, 8, A, B, 16, float("nan"), Y, None, None, 0, None, None) == 1
+    assert fwd(ctypes.byref(q), X, 8, A, B, 16, 2.0, Y, None, None, 0, None, None) == 4
+    assert fwd(ctypes.byref(q), P(0x50002), 8, A, B, 16, 2.0, Y, None, None, 0, None, None) == 3
+    q_rows = _nf4(40, 64)
+    assert fwd(ctypes.byref(q_rows), X, 8, A, B, 16, 2.0, Y, None, None, 0, None, None) == 2
+    bwd = so.qlora_linear_bwd
+    assert bwd(ctypes.byref(q), X, 8, A, B, 16, 2.0, None, None, None, P(0x90000), P(0xA0000),
+               P(0xB0000), 1 << 20, None, None) == 1
+    assert so.qlora_linear_workspace(8, 32, 64, 16, None) == 1
+    ws = SZ()
+    assert so.qlora_linear_workspace(8, 32, 100, 16, ctypes.byref(ws)) == 2
+
+
+def test_workspace_grows_with_tokens(lib):
+    small = lib.linear_workspace(64, 1024, 1024, 8)
+    big = lib.linear_workspace(2048, 4096, 4096, 16)
+    assert 0 < small < big

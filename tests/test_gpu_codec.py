@@ -1,0 +1,91 @@
+"""GPU parity of the NF4 codec against the oracle: packed codes, 8-bit block
+scales, fp32 second-level scales and the dequantised bf16 weight must be
+bit-exact ("QLoRA, in depth", "The mechanism in brief")."""
+
+import numpy as np
+import pytest
+
+from oracle import nf4 as onf4
+from bit_nf4_quantized_dequant_b200 import inputs
+
+from helpers import bf16_dev_bits
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    (1024, 1024, False),    # single linear 1024x1024
+    (4096, 4096, True),     # attention projection with 0.1% x8 outliers
+    (48, 192, False),       # 144 blocks: one short group
+    (16, 64, False),        # one block per row
+    (272, 320, True),       # ragged: 1360 blocks = 5 groups + 80
+    (11008, 128, False),    # tall
+]
+
+
+def _quantize_gpu(lib, W):
+    import torch
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    q = lib.nf4_quantize(torch.from_numpy(W).cuda(), status=status)
+    torch.cuda.synchronize()
+    return q, int(status.item())
+
+
+@pytest.mark.parametrize("N,K,outliers", SHAPES)
+def test_quantize_bit_exact(lib, N, K, outliers):
+    W = inputs.weight_f32(N, K, outliers=outliers)
+    q, st = _quantize_gpu(lib, W)
+    assert st == 0
+    codes, s8, s2 = onf4.quantize(W)
+    assert np.array_equal(q.codes.cpu().numpy(), codes)
+    assert np.array_equal(q.scale8.cpu().numpy(), s8)
+    assert np.array_equal(q.scale2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K,outliers", SHAPES)
+def test_dequantize_bit_exact(lib, N, K, outliers):
+    W = inputs.weight_f32(N, K, index=1, outliers=outliers)
+    q, _ = _quantize_gpu(lib, W)
+    out = lib.nf4_dequantize(q)
+    import torch
+    torch.cuda.synchronize()
+    codes, s8, s2 = onf4.quantize(W)
+    ref = onf4.dequantize_bits(codes, s8, s2, N, K)
+    assert np.array_equal(bf16_dev_bits(out), ref)
+
+
+def test_special_blocks(lib):
+    """All-zero blocks, signed zeros, subnormals, a block whose max is negative,
+    exact midpoint ties between levels."""
+    W = np.zeros((4, 256), dtype=np.float32)
+    W[0, 64:128] = inputs.normal_f32(9, 64, 1e-39)        # subnormal block
+    W[1, :64] = -np.abs(inputs.normal_f32(10, 64, 0.5))
+    W[1, 5] = -3.0                                         # negative absmax -> code 0
+    W[2, 64] = -0.0
+    L = onf4.nf4_levels().astype(np.float64)
+    mids = [np.float32((L[i] + L[i + 1]) / 2) for i in range(15)]
+    W[3, :15] = mids
+    W[3, 15] = 1.0
+    W[3, 64:79] = [np.nextafter(m, np.float32(2)) for m in mids]
+    W[3, 79] = -1.0
+    q, st = _quantize_gpu(lib, W)
+    assert st == 0
+    codes, s8, s2 = onf4.quantize(W)
+    assert np.array_equal(q.codes.cpu().numpy(), codes)
+    assert np.array_equal(q.scale8.cpu().numpy(), s8)
+    assert np.array_equal(q.scale2.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+    out = lib.nf4_dequantize(q)
+    assert np.array_equal(bf16_dev_bits(out), onf4.dequantize_bits(codes, s8, s2, 4, 256))
+
+
+@pytest.mark.parametrize("bad", [np.inf, -np.inf, np.nan])
+def test_nonfinite_sets_device_status(lib, bad):
+    W = inputs.weight_f32(32, 128)
+    W[7, 33] = bad
+    _, st = _quantize_gpu(lib, W)
+    assert st == 5  # QLORA_ERR_NONFINITE
+
+
+def test_status_is_cleared_by_next_quantize(lib):
+    W = inputs.weight_f32(32, 128)
+    _, st = _quantize_gpu(lib, W)
+    assert st == 0
