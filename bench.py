@@ -1,0 +1,546 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA linear layer (libqlora) on B200.
+
+One step = one training pass of the layer: forward (sU = s X A^T, then the
+fused NF4-dequant tensor-core GEMM Y = X W'^T + sU B^T) and backward
+(sT = s dY B, the fused dX = dY W' + sT A GEMM, dA = sT^T X, dB = dY^T sU),
+on the Llama-7B attention-projection workload (W 4096x4096 NF4 with 0.1% x8
+outliers, 2048 tokens, r = 16, alpha = 32). The JSON line also carries the
+standalone dequantisation bandwidth and the 8-token forward bandwidth over the
+8B linear set, the roofline of the dominant kernel, the end-to-end number
+through the public API with host buffers, the clocks seen while timing and the
+CPU oracle's throughput on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 (under torchrun) every rank runs an independent replica of
+the workload (the layer does not exchange data); the time is the maximum over
+ranks and the value counts the work of all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & NF4 dequant GB/s (1xB200, % of roofline)"
+WORKLOAD = "attn_proj_7b"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-extras", action="store_true", help="skip the 8B-set dequant / decode lines")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x20: "sync_boost", 0x40: "sw_thermal_slowdown", 0x80: "hw_thermal_slowdown",
+           0x100: "hw_power_brake_slowdown", 0x200: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._active = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        while not self._stop.is_set():
+            if self._active.is_set() and self.nv is not None:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, reasons))
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        self._active.set()
+
+    def stop(self):
+        self._active.clear()
+
+    def close(self):
+        self._stop.set()
+        self.t.join(timeout=1)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = [n for b, n in REASONS.items() if bits & b and b != 0x1]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only: the only collective is the timing max)
+# ---------------------------------------------------------------------------
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+def step_flops(M, N, K, r):
+    """Algorithmic flops of one fwd+bwd: the two dense products 2MNK each and
+    the six rank-r products 2Mr(K) or 2Mr(N) (no dW)."""
+    return 4 * M * N * K + 6 * M * r * (K + N)
+
+
+def fused_flops(mode, M, N, K, r):
+    return 2 * M * N * K + (2 * M * N * r if mode == "fwd" else 2 * M * K * r)
+
+
+def make_sets(q, torch, n_sets, N, K, M, r, outliers):
+    from bit_nf4_quantized_dequant_b200 import inputs
+    sets = []
+    for i in range(n_sets):
+        c = inputs.linear_case(N, K, M, r, index=i, outliers=outliers)
+        bf = lambda b: torch.from_numpy(b.view("int16")).view(torch.bfloat16).cuda()
+        Wf = torch.from_numpy(c["W"]).cuda()
+        nf4 = q.nf4_quantize(Wf)
+        del Wf
+        d = dict(q=nf4, X=bf(c["X"]), A=bf(c["A"]), B=bf(c["B"]), dY=bf(c["dY"]))
+        d["Y"] = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        d["dX"] = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        d["sU"] = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        d["sT"] = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        d["dA"] = torch.empty((r, K), dtype=torch.float32, device="cuda")
+        d["dB"] = torch.empty((N, r), dtype=torch.float32, device="cuda")
+        d["ws"] = torch.empty(q.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+        sets.append(d)
+    torch.cuda.synchronize()
+    return sets
+
+
+def set_bytes(M, N, K, r):
+    packed = N * K // 2 + N * K // 64 + 4 * -(-(N * K // 64) // 256)
+    return packed + 2 * (2 * M * K + 2 * M * N) + 2 * r * (K + N) + 4 * M * r + 4 * r * (K + N)
+
+
+def run_step(q, d, s, ev=None):
+    q.lora_xa(d["X"], d["A"], s, d["sU"], d["ws"])
+    if ev is not None:
+        ev[0].record()
+    q.fused_fwd(d["q"], d["X"], d["B"], d["sU"], d["Y"])
+    if ev is not None:
+        ev[1].record()
+    q.lora_dyb(d["dY"], d["B"], s, d["sT"], d["ws"])
+    if ev is not None:
+        ev[2].record()
+    q.fused_dx(d["q"], d["dY"], d["A"], d["sT"], d["dX"])
+    if ev is not None:
+        ev[3].record()
+    q.lora_grads(d["X"], d["dY"], d["sU"], d["sT"], d["dA"], d["dB"], d["ws"])
+
+
+LAUNCHES_PER_STEP = 10   # lora_xa 2, fused_fwd 1, lora_dyb 2, fused_dx 1, lora_grads 4
+
+
+def profile_traffic(kernel_file_hash):
+    """dram bytes per launch of the fused GEMM from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "fused_nf4_gemm_attn_proj_7b.md")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("kernel_source_sha256") != kernel_file_hash:
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("qlora_gemm.cu", "qlora_device.cuh"):
+        with open(os.path.join(ROOT, "bit_nf4_quantized_dequant_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------------------
+# extras on the 8B linear set: standalone dequant and the 8-token forward
+# ---------------------------------------------------------------------------
+def eight_b_set(q, torch):
+    from bit_nf4_quantized_dequant_b200 import inputs
+    wl = inputs.WORKLOADS["set_8b"]
+    g = torch.Generator(device="cuda")
+    mats = []
+    for i, lin in enumerate(wl.linears):
+        g.manual_seed(1000 + i)
+        Wf = torch.randn((lin.N, lin.K), generator=g, device="cuda", dtype=torch.float32) * 0.02
+        mats.append((lin, q.nf4_quantize(Wf)))
+        del Wf
+    torch.cuda.synchronize()
+    return mats
+
+
+def bench_dequant(q, torch, mats, steps, warmup):
+    outs = [torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device="cuda") for lin, _ in mats]
+    moved = sum(lin.N * lin.K * 2 + sum(q.nf4_sizes(lin.N, lin.K)) for lin, _ in mats)
+    for _ in range(warmup):
+        for (lin, m), o in zip(mats, outs):
+            q.nf4_dequantize(m, out=o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        for (lin, m), o in zip(mats, outs):
+            q.nf4_dequantize(m, out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del outs
+    return {"workload": "set_8b dequant: 224 matrices (32 layers x 7) to bf16", "GB/s": moved / ms / 1e6,
+            "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats)}
+
+
+def bench_decode(q, torch, mats, steps, warmup):
+    from bit_nf4_quantized_dequant_b200 import inputs
+    M, r = 8, 16
+    s = 2.0
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    per_shape = {}
+    lora = []
+    moved = 0
+    for lin, m in mats:
+        key = (lin.N, lin.K)
+        if key not in per_shape:
+            X = (torch.randn((M, lin.K), generator=g, device="cuda")).to(torch.bfloat16)
+            per_shape[key] = dict(X=X, Y=torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda"),
+                                  sU=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
+                                  ws=torch.empty(q.linear_workspace(M, lin.N, lin.K, r), dtype=torch.uint8,
+                                                 device="cuda"))
+        A = (torch.randn((r, lin.K), generator=g, device="cuda") / r).to(torch.bfloat16)
+        B = (torch.randn((lin.N, r), generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+        lora.append((A, B))
+        moved += sum(q.nf4_sizes(lin.N, lin.K)) + 2 * r * (lin.N + lin.K) + 2 * M * (lin.N + lin.K)
+
+    def one_pass():
+        for (lin, m), (A, B) in zip(mats, lora):
+            d = per_shape[(lin.N, lin.K)]
+            q.lora_xa(d["X"], A, s, d["sU"], d["ws"])
+            q.fused_fwd(m, d["X"], B, d["sU"], d["Y"])
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one_pass()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"workload": "set_8b forward at 8 tokens: 224 matrices, r=16", "GB/s": moved / ms / 1e6,
+            "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": 3 * len(mats)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (bounded sample)
+# ---------------------------------------------------------------------------
+def oracle_sample(min_seconds=10.0, max_reps=4):
+    """The oracle as it stands on one full step of the attention-projection
+    workload: dequantise W, forward and backward over all 2048 tokens."""
+    import numpy as np
+    from oracle import linear as olin, nf4 as onf4
+    from bit_nf4_quantized_dequant_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD]
+    lin = wl.linears[0]
+    N, K, M, r, s = lin.N, lin.K, wl.M, wl.r, wl.s
+    c = inputs.linear_case(N, K, M, r, outliers=True)
+    codes, s8, s2 = onf4.quantize(c["W"])
+    f = lambda b: inputs.bf16_bits_to_f32(b).astype(np.float64)
+    X, A, B, dY = f(c["X"]), f(c["A"]), f(c["B"]), f(c["dY"])
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        Wd = onf4.dequantize(codes, s8, s2, N, K)
+        olin.linear_fwd(Wd, X, A, B, s)
+        olin.linear_bwd(Wd, X, A, B, s, dY)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            break
+    try:
+        import threadpoolctl
+        cores = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas")
+    except Exception:
+        cores = os.cpu_count()
+    flops = step_flops(M, N, K, r) * reps
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} full step(s) of {WORKLOAD} (dequantise W 4096x4096, fwd+bwd over 2048 tokens) "
+                      f"in numpy float64, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return
+    import numpy as np
+    from oracle import linear as olin, nf4 as onf4
+    from bit_nf4_quantized_dequant_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD]
+    lin = wl.linears[0]
+    N, K, M, r, s = lin.N, lin.K, wl.M, wl.r, wl.s
+    Ms = 256   # tokens per reference step (a bounded sample of the 2048)
+    c = inputs.linear_case(N, K, M, r, outliers=True)
+    codes, s8, s2 = onf4.quantize(c["W"])
+    f = lambda b: inputs.bf16_bits_to_f32(b).astype(np.float64)
+    X, A, B, dY = f(c["X"]), f(c["A"]), f(c["B"]), f(c["dY"])
+
+    def one(k):
+        rows = slice((k * Ms) % M, (k * Ms) % M + Ms)
+        Wd = onf4.dequantize(codes, s8, s2, N, K)
+        olin.linear_fwd(Wd, X[rows], A, B, s)
+        olin.linear_bwd(Wd, X[rows], A, B, s, dY[rows])
+
+    steps = max(1, min(args.steps, 8))
+    for k in range(min(args.warmup, 1)):
+        one(k)
+    t0 = time.perf_counter()
+    for k in range(steps):
+        one(k)
+    el = time.perf_counter() - t0
+    flops = step_flops(Ms, N, K, r) * steps
+    val = flops / el / 1e12
+    try:
+        import threadpoolctl
+        cores = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas")
+    except Exception:
+        cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": el / steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "N": N, "K": K, "M": M, "r": r, "alpha": wl.alpha,
+                       "sample_tokens_per_step": Ms},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{steps} steps of {Ms} tokens each (dequantise W + fwd + bwd), float64"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, local = init_dist()
+    import torch
+    torch.cuda.set_device(local)
+    import bit_nf4_quantized_dequant_b200 as q
+    from bit_nf4_quantized_dequant_b200 import _build, inputs
+    if rank == 0:
+        _build.build()
+    barrier(world)
+    q.library()
+    peaks, peak_kind = load_peaks()
+
+    wl = inputs.WORKLOADS[WORKLOAD]
+    lin = wl.linears[0]
+    N, K, M, r, s = lin.N, lin.K, wl.M, wl.r, wl.s
+    per_set = set_bytes(M, N, K, r)
+    n_sets = max(2, -(-3 * L2_BYTES // per_set))
+    sets = make_sets(q, torch, n_sets, N, K, M, r, wl.outliers)
+
+    for k in range(max(3, args.warmup)):
+        run_step(q, sets[k % n_sets], s)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    K_steps = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0.record()
+    for k in range(K_steps):
+        run_step(q, sets[k % n_sets], s, evs[k])
+    e1.record()
+    torch.cuda.synchronize()
+    sampler.stop()
+    barrier(world)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = ms_total / K_steps
+    flops = step_flops(M, N, K, r)
+    value = world * flops * K_steps / (ms_total * 1e-3) / 1e12
+
+    fwd_ms = [ev[0].elapsed_time(ev[1]) for ev in evs]
+    dx_ms = [ev[2].elapsed_time(ev[3]) for ev in evs]
+    fused_total_ms = sum(fwd_ms) + sum(dx_ms)
+    fused_total_flops = K_steps * (fused_flops("fwd", M, N, K, r) + fused_flops("dx", M, N, K, r))
+    achieved = fused_total_flops / (fused_total_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    traffic = profile_traffic(kernel_source_hash())
+
+    # end to end through the public API with pinned host buffers
+    d = sets[0]
+    Xh = d["X"].cpu().pin_memory()
+    dYh = d["dY"].cpu().pin_memory()
+    Yh = torch.empty_like(d["Y"], device="cpu").pin_memory()
+    dXh = torch.empty_like(d["dX"], device="cpu").pin_memory()
+    dAh = torch.empty_like(d["dA"], device="cpu").pin_memory()
+    dBh = torch.empty_like(d["dB"], device="cpu").pin_memory()
+    Xd, dYd = torch.empty_like(d["X"]), torch.empty_like(d["dY"])
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        dYd.copy_(dYh, non_blocking=True)
+        q.linear_fwd(d["q"], Xd, d["A"], d["B"], s, Y=d["Y"], sU=d["sU"], ws=d["ws"])
+        q.linear_bwd(d["q"], Xd, d["A"], d["B"], s, dYd, sU=d["sU"], dX=d["dX"], dA=d["dA"], dB=d["dB"],
+                     ws=d["ws"])
+        Yh.copy_(d["Y"], non_blocking=True)
+        dXh.copy_(d["dX"], non_blocking=True)
+        dAh.copy_(d["dA"], non_blocking=True)
+        dBh.copy_(d["dB"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(10, K_steps // 4)
+    barrier(world)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), world) / e2e_steps
+    h2d = Xh.numel() * 2 + dYh.numel() * 2
+    d2h = Yh.numel() * 2 + dXh.numel() * 2 + dAh.numel() * 4 + dBh.numel() * 4
+
+    extras = {}
+    if not args.no_extras:
+        del sets
+        torch.cuda.empty_cache()
+        mats = eight_b_set(q, torch)
+        extras["dequant"] = bench_dequant(q, torch, mats, steps=5, warmup=2)
+        extras["dequant"]["frac_of_hbm"] = extras["dequant"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
+        extras["decode_fwd"] = bench_decode(q, torch, mats, steps=5, warmup=2)
+        extras["decode_fwd"]["frac_of_hbm"] = extras["decode_fwd"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
+        del mats
+    sampler.close()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K_steps,
+            "warmup": max(3, args.warmup),
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "N": N, "K": K, "M": M, "r": r, "alpha": wl.alpha,
+                       "outliers": "0.1% of W x8", "flops_per_step": flops,
+                       "l2": f"inputs rotate over {n_sets} sets of {per_set/1e6:.0f} MB (> L2)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"kernel": "fused_nf4_gemm_kernel (fwd and dX launches)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": f"{peak_kind} bf16 burst", "traffic": traffic,
+                         "launch_ms_fwd": statistics.mean(fwd_ms), "launch_ms_dx": statistics.mean(dx_ms),
+                         "share_of_step": fused_total_ms / (ms_step * K_steps)},
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": LAUNCHES_PER_STEP * K_steps,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+        }
+        line.update(extras)
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -17,6 +17,7 @@ __all__ = [
     "QloraError", "QloraUnavailable", "NF4Matrix", "library", "library_path", "SYMBOLS",
     "nf4_sizes", "nf4_codebook", "nf4_quantize", "nf4_dequantize",
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
+    "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +33,7 @@ STATUS = {
 SYMBOLS = [
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_nf4_quantize", "qlora_nf4_dequantize",
     "qlora_linear_workspace", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
+    "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
 ]
 
 
@@ -84,6 +86,16 @@ def library():
     lib.qlora_linear_bwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, _P, ctypes.c_int32, ctypes.c_float,
                                      _P, _P, _P, _P, _P, _P, _SZ, _P, _P]
     lib.qlora_linear_bwd.restype = st
+    lib.qlora_lora_xa.argtypes = [_P, _I64, _I64, _P, ctypes.c_int32, ctypes.c_float, _P, _P, _SZ, _P]
+    lib.qlora_lora_xa.restype = st
+    lib.qlora_lora_dyb.argtypes = [_P, _I64, _I64, _P, ctypes.c_int32, ctypes.c_float, _P, _P, _SZ, _P]
+    lib.qlora_lora_dyb.restype = st
+    lib.qlora_fused_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P]
+    lib.qlora_fused_fwd.restype = st
+    lib.qlora_fused_dx.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P]
+    lib.qlora_fused_dx.restype = st
+    lib.qlora_lora_grads.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P]
+    lib.qlora_lora_grads.restype = st
     lib.qlora_status_string.argtypes = [ctypes.c_int]
     lib.qlora_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -215,3 +227,47 @@ def linear_bwd(q: NF4Matrix, X, A, B, s: float, dY, sU=None, dX=None, dA=None, d
                                       _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _ptr(status),
                                       _stream(stream)), "qlora_linear_bwd")
     return dX, dA, dB
+
+
+# ---- the individual steps of the layer ---------------------------------------
+
+def lora_xa(X, A, s: float, sU, ws, stream=None):
+    """sU = bf16(s X A^T)."""
+    M, K = X.shape
+    _check(library().qlora_lora_xa(_ptr(X), M, K, _ptr(A), A.shape[0], s, _ptr(sU), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "qlora_lora_xa")
+    return sU
+
+
+def lora_dyb(dY, B, s: float, sT, ws, stream=None):
+    """sT = bf16(s dY B)."""
+    M, N = dY.shape
+    _check(library().qlora_lora_dyb(_ptr(dY), M, N, _ptr(B), B.shape[1], s, _ptr(sT), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "qlora_lora_dyb")
+    return sT
+
+
+def fused_fwd(q: NF4Matrix, X, B, sU, Y, status=None, stream=None):
+    """Y = X W'^T + sU B^T (dequantisation fused into the tensor-core GEMM)."""
+    st = q.c_struct()
+    _check(library().qlora_fused_fwd(ctypes.byref(st), _ptr(X), X.shape[0], _ptr(B), B.shape[1], _ptr(sU),
+                                     _ptr(Y), _ptr(status), _stream(stream)), "qlora_fused_fwd")
+    return Y
+
+
+def fused_dx(q: NF4Matrix, dY, A, sT, dX, status=None, stream=None):
+    """dX = dY W' + sT A (dequantisation fused into the tensor-core GEMM)."""
+    st = q.c_struct()
+    _check(library().qlora_fused_dx(ctypes.byref(st), _ptr(dY), dY.shape[0], _ptr(A), A.shape[0], _ptr(sT),
+                                    _ptr(dX), _ptr(status), _stream(stream)), "qlora_fused_dx")
+    return dX
+
+
+def lora_grads(X, dY, sU, sT, dA, dB, ws, stream=None):
+    """dA = sT^T X, dB = dY^T sU (fp32, overwritten)."""
+    M, K = X.shape
+    N = dY.shape[1]
+    r = sU.shape[1]
+    _check(library().qlora_lora_grads(_ptr(X), _ptr(dY), M, N, K, _ptr(sU), _ptr(sT), r, _ptr(dA), _ptr(dB),
+                                      _ptr(ws), ws.numel(), _stream(stream)), "qlora_lora_grads")
+    return dA, dB

@@ -156,6 +156,83 @@ qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r
   return QLORA_OK;
 }
 
+qlora_status_t qlora_lora_xa(const uint16_t *X, int64_t M, int64_t K, const uint16_t *A, int32_t r,
+                             float s, uint16_t *sU, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!X || !A || !sU || M <= 0 || K <= 0 || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (K % kBlock || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(sU) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
+  const size_t need = lora_rows_ws_floats(M, K, r) * 4;
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  return cuda_status(launch_lora_rows(X, M, K, A, r, /*w_is_rk=*/true, s, sU, static_cast<float *>(ws),
+                                      ws_bytes / 4, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const uint16_t *B, int32_t r,
+                              float s, uint16_t *sT, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!dY || !B || !sT || M <= 0 || N <= 0 || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(dY) || !aligned16(B) || !aligned16(sT) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
+  const size_t need = lora_rows_ws_floats(M, N, r) * 4;
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  return cuda_status(launch_lora_rows(dY, M, N, B, r, /*w_is_rk=*/false, s, sT, static_cast<float *>(ws),
+                                      ws_bytes / 4, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act, int64_t M,
+                            const uint16_t *lora_w, int32_t r, const uint16_t *lora_act, uint16_t *out,
+                            int32_t *dev_status, qlora_stream_t stream) {
+  qlora_status_t st = check_linear(W, act, M, lora_w, lora_w, r, 1.0f);
+  if (st != QLORA_OK) return st;
+  if (!lora_act || !out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(lora_act) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
+  GemmArgs g{};
+  g.mode = mode;
+  g.codes = W->codes;
+  g.scale8 = W->scale8;
+  g.scale2 = W->scale2;
+  g.N = W->rows;
+  g.K = W->cols;
+  g.M = M;
+  g.r = r;
+  g.act = act;
+  g.lora_w = lora_w;
+  g.lora_act = lora_act;
+  g.out = out;
+  g.dev_status = dev_status;
+  return cuda_status(launch_fused_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_fused_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *B,
+                               int32_t r, const uint16_t *sU, uint16_t *Y, int32_t *dev_status,
+                               qlora_stream_t stream) {
+  return fused(0, W, X, M, B, r, sU, Y, dev_status, stream);
+}
+
+qlora_status_t qlora_fused_dx(const qlora_nf4_t *W, const uint16_t *dY, int64_t M, const uint16_t *A,
+                              int32_t r, const uint16_t *sT, uint16_t *dX, int32_t *dev_status,
+                              qlora_stream_t stream) {
+  return fused(1, W, dY, M, A, r, sT, dX, dev_status, stream);
+}
+
+qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                                const uint16_t *sU, const uint16_t *sT, int32_t r, float *dA, float *dB,
+                                void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!X || !dY || !sU || !sT || !dA || !dB || M <= 0 || N <= 0 || K <= 0) return QLORA_ERR_INVALID_ARG;
+  if (K % kBlock || N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(sU) || !aligned16(sT) || !aligned16(dA) ||
+      !aligned16(dB) || (ws && !aligned16(ws)))
+    return QLORA_ERR_MISALIGNED;
+  const size_t fa = lora_cols_ws_floats(M, K, r), fb = lora_cols_ws_floats(M, N, r);
+  if (!ws || ws_bytes < 4 * (fa > fb ? fa : fb)) return QLORA_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  float *part = static_cast<float *>(ws);
+  // dA[j, k] = sum_m sT[m, j] X[m, k];  dB[n, j] = sum_m dY[m, n] sU[m, j]
+  cudaError_t e = launch_lora_cols(X, M, K, sT, r, /*transpose_out=*/true, dA, part, ws_bytes / 4, cs);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  return cuda_status(launch_lora_cols(dY, M, N, sU, r, /*transpose_out=*/false, dB, part, ws_bytes / 4, cs));
+}
+
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
                                 void *ws, size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
@@ -167,28 +244,11 @@ qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   const WsLayout L = ws_layout(M, N, K, r);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(wsb + L.su);
-  float *part = reinterpret_cast<float *>(wsb + L.part);
-
-  cudaError_t e = launch_lora_rows(X, M, K, A, r, /*w_is_rk=*/true, s, sU, part, L.part_floats, cs);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  GemmArgs g{};
-  g.mode = 0;
-  g.codes = W->codes;
-  g.scale8 = W->scale8;
-  g.scale2 = W->scale2;
-  g.N = N;
-  g.K = K;
-  g.M = M;
-  g.r = r;
-  g.act = X;
-  g.lora_w = B;
-  g.lora_act = sU;
-  g.out = Y;
-  g.dev_status = dev_status;
-  return cuda_status(launch_fused_gemm(g, cs));
+  st = qlora_lora_xa(X, M, K, A, r, s, sU, wsb + L.part, L.part_floats * 4, stream);
+  if (st != QLORA_OK) return st;
+  return qlora_fused_fwd(W, X, M, B, r, sU, Y, dev_status, stream);
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
@@ -205,44 +265,24 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   const WsLayout L = ws_layout(M, N, K, r);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   uint16_t *sT = reinterpret_cast<uint16_t *>(wsb + L.st);
-  float *part = reinterpret_cast<float *>(wsb + L.part);
+  void *part = wsb + L.part;
+  const size_t part_bytes = L.part_floats * 4;
   const uint16_t *sU = sU_in;
-  cudaError_t e;
   if (!sU) {
     uint16_t *su_ws = reinterpret_cast<uint16_t *>(wsb + L.su);
-    e = launch_lora_rows(X, M, K, A, r, true, s, su_ws, part, L.part_floats, cs);
-    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    st = qlora_lora_xa(X, M, K, A, r, s, su_ws, part, part_bytes, stream);
+    if (st != QLORA_OK) return st;
     sU = su_ws;
   }
-  // sT = bf16(s * dY B)
-  e = launch_lora_rows(dY, M, N, B, r, /*w_is_rk=*/false, s, sT, part, L.part_floats, cs);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  st = qlora_lora_dyb(dY, M, N, B, r, s, sT, part, part_bytes, stream);
+  if (st != QLORA_OK) return st;
   if (dX) {
-    GemmArgs g{};
-    g.mode = 1;
-    g.codes = W->codes;
-    g.scale8 = W->scale8;
-    g.scale2 = W->scale2;
-    g.N = N;
-    g.K = K;
-    g.M = M;
-    g.r = r;
-    g.act = dY;
-    g.lora_w = A;
-    g.lora_act = sT;
-    g.out = dX;
-    g.dev_status = dev_status;
-    e = launch_fused_gemm(g, cs);
-    if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    st = qlora_fused_dx(W, dY, M, A, r, sT, dX, dev_status, stream);
+    if (st != QLORA_OK) return st;
   }
-  // dA[j, k] = sum_m sT[m, j] X[m, k];  dB[n, j] = sum_m dY[m, n] sU[m, j]
-  e = launch_lora_cols(X, M, K, sT, r, /*transpose_out=*/true, dA, part, L.part_floats, cs);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  e = launch_lora_cols(dY, M, N, sU, r, /*transpose_out=*/false, dB, part, L.part_floats, cs);
-  return cuda_status(e);
+  return qlora_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, part, part_bytes, stream);
 }
 
 const char *qlora_status_string(qlora_status_t status) {

@@ -143,6 +143,48 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
                                 float *dA, float *dB, void *ws, size_t ws_bytes,
                                 int32_t *dev_status, qlora_stream_t stream);
 
+/*
+ * The five steps of the layer, one entry point each. qlora_linear_fwd runs
+ * qlora_lora_xa then qlora_fused_fwd; qlora_linear_bwd runs qlora_lora_dyb,
+ * qlora_fused_dx and qlora_lora_grads (and qlora_lora_xa when sU is not
+ * given). They are exposed so that a caller can schedule or time the steps
+ * separately; arguments, layouts and errors are as in the composite calls.
+ * `ws` is a workspace of at least qlora_linear_workspace() bytes for the same
+ * (M, N, K, r); it only holds partial sums between the two kernels of a step.
+ */
+
+/* sU = bf16_rn(s X A^T), [M, r]. The adapter's down projection, the first
+ * half of (alpha / r) B A x ("QLoRA, in depth", "The mechanism in brief").
+ * K % 64 == 0. Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
+qlora_status_t qlora_lora_xa(const uint16_t *X, int64_t M, int64_t K, const uint16_t *A, int32_t r,
+                             float s, uint16_t *sU, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Y = X W'^T + sU B^T with W' dequantised tile by tile in shared memory and
+ * fed to the tensor cores; the LoRA term is one extra K-step of the same
+ * accumulation ("QLoRA and Fine-Tuning on One Consumer GPU", "The idea in one
+ * line"). Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+qlora_status_t qlora_fused_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *B,
+                               int32_t r, const uint16_t *sU, uint16_t *Y, int32_t *dev_status,
+                               qlora_stream_t stream);
+
+/* sT = bf16_rn(s dY B), [M, r]: the gradient reaching the adapter's
+ * bottleneck. N % 16 == 0. Errors: as qlora_lora_xa. */
+qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const uint16_t *B, int32_t r,
+                              float s, uint16_t *sT, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* dX = dY W' + sT A, [M, K] bf16, W' dequantised in shared memory as in
+ * qlora_fused_fwd (here consumed untransposed). Errors: as qlora_fused_fwd. */
+qlora_status_t qlora_fused_dx(const qlora_nf4_t *W, const uint16_t *dY, int64_t M, const uint16_t *A,
+                              int32_t r, const uint16_t *sT, uint16_t *dX, int32_t *dev_status,
+                              qlora_stream_t stream);
+
+/* dA = sT^T X ([r, K] fp32) and dB = dY^T sU ([N, r] fp32), both overwritten:
+ * the adapter gradients ("QLoRA, in depth", "The mechanism in brief").
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
+qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                                const uint16_t *sU, const uint16_t *sT, int32_t r, float *dA, float *dB,
+                                void *ws, size_t ws_bytes, qlora_stream_t stream);
+
 /* A static, human-readable name for a status code (host). */
 const char *qlora_status_string(qlora_status_t status);
 
