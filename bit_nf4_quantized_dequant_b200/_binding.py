@@ -17,7 +17,7 @@ __all__ = [
     "QloraError", "QloraUnavailable", "NF4Matrix", "library", "library_path", "SYMBOLS",
     "nf4_sizes", "nf4_codebook", "nf4_quantize", "nf4_dequantize",
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
-    "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads",
+    "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +34,7 @@ SYMBOLS = [
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_nf4_quantize", "qlora_nf4_dequantize",
     "qlora_linear_workspace", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
+    "qlora_linear_fwd_noalloc",
 ]
 
 
@@ -96,6 +97,9 @@ def library():
     lib.qlora_fused_dx.restype = st
     lib.qlora_lora_grads.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P]
     lib.qlora_lora_grads.restype = st
+    lib.qlora_linear_fwd_noalloc.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, _P, ctypes.c_int32,
+                                             ctypes.c_float, _P, _P, _P, _P]
+    lib.qlora_linear_fwd_noalloc.restype = st
     lib.qlora_status_string.argtypes = [ctypes.c_int]
     lib.qlora_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -271,3 +275,17 @@ def lora_grads(X, dY, sU, sT, dA, dB, ws, stream=None):
     _check(library().qlora_lora_grads(_ptr(X), _ptr(dY), M, N, K, _ptr(sU), _ptr(sT), r, _ptr(dA), _ptr(dB),
                                       _ptr(ws), ws.numel(), _stream(stream)), "qlora_lora_grads")
     return dA, dB
+
+
+def linear_fwd_noalloc(q: NF4Matrix, X, A, B, s: float, Y=None, sU=None, status=None, stream=None):
+    """Y = X W'^T + s (X A^T) B^T without a workspace: the library takes its
+    scratch from a fixed device array (see qlora_linear_fwd_noalloc)."""
+    import torch
+    M = X.shape[0]
+    r = A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    st = q.c_struct()
+    _check(library().qlora_linear_fwd_noalloc(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y),
+                                              _ptr(sU), _ptr(status), _stream(stream)), "qlora_linear_fwd_noalloc")
+    return Y, sU

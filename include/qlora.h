@@ -185,6 +185,34 @@ qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M
                                 const uint16_t *sU, const uint16_t *sT, int32_t r, float *dA, float *dB,
                                 void *ws, size_t ws_bytes, qlora_stream_t stream);
 
+/*
+ * Allocation-free forward. The pages have no counterpart to this call: it is an
+ * interface convenience of this library for callers that cannot allocate
+ * device memory where they run the layer (a plug-in that only receives its
+ * inputs and outputs, a server whose device memory is all handed to a fixed
+ * pool up front, code that must not call cudaMalloc between launches because
+ * that call can synchronise the device).
+ * It computes exactly what qlora_linear_fwd computes, with the same arguments
+ * minus the workspace: its scratch (the split-K partial sums of s X A^T, plus
+ * sU itself when sU_out is NULL) lives in one 8 MiB array compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits. It calls no allocator.
+ * Limit: round_up(M*r*2, 256) (only when sU_out is NULL) + the partial sums
+ * (4 * splits * M * r bytes, splits <= 2 * SM count / ceil(M/64)) must fit in
+ * 8 MiB; larger calls return QLORA_ERR_WORKSPACE before anything is launched.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. Every call shares the one array and leaves its contents
+ * behind; nothing in it needs to start at zero, but calls whose kernels can
+ * overlap on the GPU (other streams, other host threads) race on it, so the
+ * caller must serialise them.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA.
+ */
+qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const uint16_t *X, int64_t M,
+                                        const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                                        uint16_t *Y, uint16_t *sU_out, int32_t *dev_status,
+                                        qlora_stream_t stream);
+
 /* A static, human-readable name for a status code (host). */
 const char *qlora_status_string(qlora_status_t status);
 
