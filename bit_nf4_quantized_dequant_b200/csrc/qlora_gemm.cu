@@ -96,6 +96,45 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmParams &p) {
   return s;
 }
 
+// Slot and phase of a ring position, advanced without division.
+struct RingPos {
+  int slot;
+  uint32_t phase;
+  __device__ __forceinline__ void advance(int by, int slots) {
+    slot += by;
+    while (slot >= slots) {
+      slot -= slots;
+      phase ^= 1u;
+    }
+  }
+};
+
+// (local tile, k-step) of a position in this CTA's step sequence, advanced
+// without division; rt is the tile's index along the UMMA M dimension.
+struct StepPos {
+  int lt, k, rt, tt;
+  __device__ __forceinline__ void set_tile(int row_tiles) {
+    const int tile = static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x);
+    rt = tile % row_tiles;
+    tt = tile / row_tiles;
+  }
+  __device__ __forceinline__ void init(int it, int nk, int row_tiles) {
+    lt = it / nk;
+    k = it - lt * nk;
+    set_tile(row_tiles);
+  }
+  __device__ __forceinline__ void advance(int by, int nk, int row_tiles) {
+    k += by;
+    if (k >= nk) {
+      while (k >= nk) {
+        k -= nk;
+        ++lt;
+      }
+      set_tile(row_tiles);
+    }
+  }
+};
+
 // Number of tiles this CTA processes (tiles blockIdx.x, blockIdx.x + gridDim.x, ...).
 __device__ __forceinline__ int local_tiles(int ntiles) {
   const int b = static_cast<int>(blockIdx.x), g = static_cast<int>(gridDim.x);
@@ -167,16 +206,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       uint32_t mask = 0, par = 0;
       bool ok = true;
-      for (int it = 0; it < total_steps; ++it) {
-        const int lt = it / p.nk, k = it - lt * p.nk;
-        const int rt = (static_cast<int>(blockIdx.x) + lt * grid) % p.row_tiles;
-        const int s = it % p.sc;
-        const uint32_t ph = static_cast<uint32_t>(it / p.sc) & 1u;
+      RingPos c{0, 0};
+      StepPos sp;
+      sp.init(0, p.nk, p.row_tiles);
+      for (int it = 0; it < total_steps; ++it, c.advance(1, p.sc), sp.advance(1, p.nk, p.row_tiles)) {
+        const int s = c.slot;
+        const uint32_t ph = c.phase;
         if (!mbar_wait(&sm.ce[s], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
         mbar_arrive_expect_tx(&sm.cf[s], kCodeTileBytes);
-        uint8_t *c = sm.c + static_cast<size_t>(s) * kCodeTileBytes;
-        if (!dx) tma_load_2d(c, &tm_codes, &sm.cf[s], k * (kKStage / 2), rt * kTileRows);
-        else     tma_load_2d(c, &tm_codes, &sm.cf[s], rt * (kTileRows / 2), k * kKStage);
+        uint8_t *cp = sm.c + static_cast<size_t>(s) * kCodeTileBytes;
+        if (!dx) tma_load_2d(cp, &tm_codes, &sm.cf[s], sp.k * (kKStage / 2), sp.rt * kTileRows);
+        else     tma_load_2d(cp, &tm_codes, &sm.cf[s], sp.rt * (kTileRows / 2), sp.k * kKStage);
         mask |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       }
@@ -187,14 +227,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       uint32_t mask = 0, par = 0;
       bool ok = true;
-      for (int it = 0; it < total_steps; ++it) {
-        const int lt = it / p.nk, k = it - lt * p.nk;
-        const int tt = (static_cast<int>(blockIdx.x) + lt * grid) / p.row_tiles;
-        const int s = it % p.sx;
-        const uint32_t ph = static_cast<uint32_t>(it / p.sx) & 1u;
+      RingPos x{0, 0};
+      StepPos sp;
+      sp.init(0, p.nk, p.row_tiles);
+      for (int it = 0; it < total_steps; ++it, x.advance(1, p.sx), sp.advance(1, p.nk, p.row_tiles)) {
+        const int s = x.slot;
+        const uint32_t ph = x.phase;
         if (!mbar_wait(&sm.xe[s], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
         mbar_arrive_expect_tx(&sm.xf[s], sm.x_bytes);
-        tma_load_2d(sm.x + static_cast<size_t>(s) * sm.x_bytes, &tm_act, &sm.xf[s], k * kKStage, tt * p.bt);
+        tma_load_2d(sm.x + static_cast<size_t>(s) * sm.x_bytes, &tm_act, &sm.xf[s], sp.k * kKStage, sp.tt * p.bt);
         mask |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       }
@@ -231,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lsbo = 16u * static_cast<uint32_t>(p.r_pad);   // 8 rows of 2 r_pad bytes
       const uint32_t la_addr = smem_u32(sm.la), lb_addr = smem_u32(sm.lb);
       bool ok = true, issued_any = false;
-      int it = 0;
+      RingPos xr{0, 0}, ar{0, 0};
       for (int lt = 0; lt < nlt && ok; ++lt) {
         const int buf = lt & 1;
         if (!mbar_wait(&sm.acce[buf], (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
@@ -240,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * p.bt);
-        for (int k = 0; k < p.nk; ++k, ++it) {
-          const int xs = it % p.sx, as = it % p.sa;
-          if (!mbar_wait(&sm.xf[xs], static_cast<uint32_t>(it / p.sx) & 1u, abort_flag, p.status) ||
-              !mbar_wait(&sm.af[as], static_cast<uint32_t>(it / p.sa) & 1u, abort_flag, p.status)) {
+        for (int k = 0; k < p.nk; ++k, xr.advance(1, p.sx), ar.advance(1, p.sa)) {
+          const int xs = xr.slot, as = ar.slot;
+          if (!mbar_wait(&sm.xf[xs], xr.phase, abort_flag, p.status) ||
+              !mbar_wait(&sm.af[as], ar.phase, abort_flag, p.status)) {
             ok = false;
             break;
           }
@@ -336,37 +377,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t out_row = dx ? static_cast<uint32_t>(kb_loc * 8192 + (n_loc >> 3) * 1024 + (n_loc & 7) * 128)
                                 : static_cast<uint32_t>((n_loc >> 3) * 1024 + (n_loc & 7) * 128);
     const uint32_t sw = static_cast<uint32_t>(n_loc & 7);
-    // scale of this thread's block at global step `it` (q8 = 0 outside the matrix)
-    auto scale_at = [&](int it, uint32_t &q8, float &d) {
+    // scale of this thread's block at step position sp (q8 = 0 outside the matrix)
+    auto scale_at = [&](const StepPos &sp, int it, uint32_t &q8, float &d) {
       q8 = 0;
       d = 0.f;
       if (it >= total_steps) return;
-      const int lt = it / p.nk, k = it - lt * p.nk;
-      const int rt = (static_cast<int>(blockIdx.x) + lt * grid) % p.row_tiles;
       int64_t n, kb;
-      if (!dx) { n = static_cast<int64_t>(rt) * kTileRows + n_loc; kb = k; }
-      else     { n = static_cast<int64_t>(k) * kKStage + n_loc; kb = static_cast<int64_t>(rt) * 2 + kb_loc; }
+      if (!dx) { n = static_cast<int64_t>(sp.rt) * kTileRows + n_loc; kb = sp.k; }
+      else     { n = static_cast<int64_t>(sp.k) * kKStage + n_loc; kb = static_cast<int64_t>(sp.rt) * 2 + kb_loc; }
       if (n < p.N && kb < kb_row) {
         const int64_t b = n * kb_row + kb;
         q8 = __ldg(p.scale8 + b);
         d = __ldg(p.scale2 + (b >> 8));
       }
     };
-    // Scale loads run three of this group's steps ahead; the loop is unrolled
-    // by three so each prefetched value stays in its own register until used.
+    // Scale loads run three of this group's steps (six steps) ahead; the loop
+    // is unrolled by three so each prefetched value stays in its own register
+    // until it is used.
     uint32_t qv[3];
     float dv[3];
+    StepPos pf;                    // position of the next prefetch
+    pf.init(g, p.nk, p.row_tiles);
 #pragma unroll
-    for (int u = 0; u < 3; ++u) scale_at(2 * u + g, qv[u], dv[u]);
+    for (int u = 0; u < 3; ++u) {
+      scale_at(pf, 2 * u + g, qv[u], dv[u]);
+      pf.advance(2, p.nk, p.row_tiles);
+    }
+    RingPos cr{g, 0}, ar{g, 0};    // rings of depth >= 2: step g sits in slot g of phase 0
     bool ok = true;
     for (int j0 = 0; ok; j0 += 3) {
 #pragma unroll
       for (int u = 0; u < 3; ++u) {
         const int it = 2 * (j0 + u) + g;
         if (it >= total_steps) { ok = false; break; }
-        const int cs = it % p.sc, as = it % p.sa;
-        if (!mbar_wait(&sm.cf[cs], static_cast<uint32_t>(it / p.sc) & 1u, abort_flag, p.status) ||
-            !mbar_wait(&sm.ae[as], (static_cast<uint32_t>(it / p.sa) & 1u) ^ 1u, abort_flag, p.status)) {
+        const int cs = cr.slot, as = ar.slot;
+        if (!mbar_wait(&sm.cf[cs], cr.phase, abort_flag, p.status) ||
+            !mbar_wait(&sm.ae[as], ar.phase ^ 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -389,7 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.af[as]);
-        scale_at(it + 6, qv[u], dv[u]);
+        scale_at(pf, it + 6, qv[u], dv[u]);
+        pf.advance(2, p.nk, p.row_tiles);
+        cr.advance(2, p.sc);
+        ar.advance(2, p.sa);
       }
     }
   }
