@@ -162,7 +162,7 @@ qlora_status_t qlora_lora_xa(const uint16_t *X, int64_t M, int64_t K, const uint
   if (K % kBlock || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(X) || !aligned16(A) || !aligned16(sU) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
   const size_t need = lora_rows_ws_floats(M, K, r) * 4;
-  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (need > 0 && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   return cuda_status(launch_lora_rows(X, M, K, A, r, /*w_is_rk=*/true, s, sU, static_cast<float *>(ws),
                                       ws_bytes / 4, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -173,7 +173,7 @@ qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const ui
   if (N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(dY) || !aligned16(B) || !aligned16(sT) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
   const size_t need = lora_rows_ws_floats(M, N, r) * 4;
-  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (need > 0 && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   return cuda_status(launch_lora_rows(dY, M, N, B, r, /*w_is_rk=*/false, s, sT, static_cast<float *>(ws),
                                       ws_bytes / 4, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -224,7 +224,8 @@ qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M
       !aligned16(dB) || (ws && !aligned16(ws)))
     return QLORA_ERR_MISALIGNED;
   const size_t fa = lora_cols_ws_floats(M, K, r), fb = lora_cols_ws_floats(M, N, r);
-  if (!ws || ws_bytes < 4 * (fa > fb ? fa : fb)) return QLORA_ERR_WORKSPACE;
+  const size_t need = 4 * (fa > fb ? fa : fb);
+  if (need > 0 && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   float *part = static_cast<float *>(ws);
   // dA[j, k] = sum_m sT[m, j] X[m, k];  dB[n, j] = sum_m dY[m, n] sU[m, j]

@@ -1,344 +1,403 @@
 // Skinny LoRA products of the QLoRA linear ("QLoRA, in depth", section "The
 // mechanism in brief": the adapter path (alpha / r) B A x; backward gives the
 // gradients of A and B). With rank r <= 64 these are thin, memory-bound
-// reductions:
+// reductions over a long dimension:
 //   rows:  out[m, j]  = bf16_rn(s * sum_k Z[m, k] Wl(j, k))   (sU = s X A^T, sT = s dY B)
 //   cols:  out(d, j)  = sum_m Z[m, d] V[m, j]                  (dA = sT^T X, dB = dY^T sU)
-// "rows" runs on the warp-level bf16 tensor-core MMA (m16n8k16) with the
-// adapter weight staged in shared memory; "cols" accumulates in registers with
-// packed fp32x2 FMAs. Both split the reduction over CTAs, write fp32 partial
-// sums to the caller's workspace and reduce them in a fixed order in a second
-// kernel, so results are deterministic.
+// Both stream Z through a TMA ring (one producer thread keeps several 8-16 KiB
+// tiles in flight per CTA), build bf16 tensor-core fragments with ldmatrix and
+// accumulate with the warp-level MMA (m16n8k16, fp32). The reduction dimension
+// is split over the CTAs of one thread-block cluster; each CTA leaves its fp32
+// partial tile in shared memory and the cluster adds the partials through
+// distributed shared memory in rank order, so no scratch memory is used and
+// the result is deterministic.
+#include <cuda.h>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
 namespace {
 
-// ---------------------------------------------------------------------------
-// rows: Z[M, K] (bf16) x Wl(j, k) -> part[split][M][r] (fp32)
-// ---------------------------------------------------------------------------
-constexpr int kRowsWarps = 4;
-constexpr int kRowsTile = 16 * kRowsWarps;   // rows per CTA
-constexpr int kKC = 256;                     // k per staged chunk
-constexpr int kKCPad = kKC + 8;              // smem row pitch (bf16), conflict-free fragment reads
+constexpr int kStages = 6;
+constexpr int kClusterMax = 8;
+constexpr uint32_t kSpanZ = 128;   // Z tiles: 64 bf16 per row, SWIZZLE_128B
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+CUtensorMapSwizzle swizzle_for_span(int span) {
+  return span == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                    : (span == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-__device__ __forceinline__ uint32_t ldg_u32(const uint16_t *p) {
-  return __ldg(reinterpret_cast<const unsigned int *>(p));
-}
-
-template <int NT>  // n-tiles of 8 adapter columns: r_pad = 8 * NT
-__global__ void __launch_bounds__(32 * kRowsWarps) lora_rows_mma(const uint16_t *__restrict__ Z, int64_t M,
-                                                                  int64_t K, const uint16_t *__restrict__ W,
-                                                                  int r, int w_is_rk, int64_t k_per_split,
-                                                                  float *__restrict__ part) {
-  __shared__ __align__(16) uint16_t ws[NT * 8][kKCPad];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kRowsTile + warp * 16;
-  const int64_t kbeg = static_cast<int64_t>(blockIdx.y) * k_per_split;
-  const int64_t kend = min(K, kbeg + k_per_split);
-  const int64_t ra = m0 + g, rb = m0 + g + 8;
-  const bool va = ra < M, vb = rb < M;
-  const uint16_t *za = Z + (va ? ra : 0) * K;
-  const uint16_t *zb = Z + (vb ? rb : 0) * K;
-  float acc[NT][4];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-  for (int64_t k0 = kbeg; k0 < kend; k0 += kKC) {
-    const int kc = static_cast<int>(kend - k0 < kKC ? kend - k0 : kKC);
-    // stage the adapter weight chunk as [j][k] (bf16), zero beyond r and kend
-    for (int e = threadIdx.x; e < NT * 8 * (kKC / 8); e += blockDim.x) {
-      const int j = e / (kKC / 8), kk = (e % (kKC / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (j < r && kk < kc) {
-        if (w_is_rk) {
-          if (kk + 8 <= kc) {
-            v = __ldg(reinterpret_cast<const uint4 *>(W + static_cast<int64_t>(j) * K + k0 + kk));
-          } else {
-            uint16_t t8[8];
-            for (int q = 0; q < 8; ++q) t8[q] = (kk + q < kc) ? W[static_cast<int64_t>(j) * K + k0 + kk + q] : 0;
-            v = *reinterpret_cast<uint4 *>(t8);
-          }
-        } else {
-          uint16_t t8[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) t8[q] = (kk + q < kc) ? W[(k0 + kk + q) * r + j] : 0;
-          v = *reinterpret_cast<uint4 *>(t8);
-        }
-      }
-      *reinterpret_cast<uint4 *>(&ws[j][kk]) = v;
-    }
-    __syncthreads();
-    const int nsteps = (kc + 15) / 16;
-    // Loads of eight k-steps are issued before their MMAs so that each lane
-    // keeps 32 independent loads in flight.
-    for (int s0 = 0; s0 < nsteps; s0 += 8) {
-      uint32_t a[8][4];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int kk = (s0 + u) * 16;
-        const int64_t kg = k0 + kk;
-        if (kk + 16 <= kc) {
-          a[u][0] = va ? ldg_u32(za + kg + 2 * c) : 0u;
-          a[u][1] = vb ? ldg_u32(zb + kg + 2 * c) : 0u;
-          a[u][2] = va ? ldg_u32(za + kg + 2 * c + 8) : 0u;
-          a[u][3] = vb ? ldg_u32(zb + kg + 2 * c + 8) : 0u;
-        } else if (kk < kc) {
-          // ragged tail of the reduction (only when kend is not a multiple of 16)
-          auto pick = [&](const uint16_t *zr, bool v, int col) -> uint32_t {
-            uint32_t lo = (v && kk + col < kc) ? zr[kg + col] : 0u;
-            uint32_t hi = (v && kk + col + 1 < kc) ? zr[kg + col + 1] : 0u;
-            return lo | (hi << 16);
-          };
-          a[u][0] = pick(za, va, 2 * c);
-          a[u][1] = pick(zb, vb, 2 * c);
-          a[u][2] = pick(za, va, 2 * c + 8);
-          a[u][3] = pick(zb, vb, 2 * c + 8);
-        } else {
-          a[u][0] = a[u][1] = a[u][2] = a[u][3] = 0u;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int kk = (s0 + u) * 16;
-        if (kk < kc) {
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const uint32_t b0 = *reinterpret_cast<const uint32_t *>(&ws[t * 8 + g][kk + 2 * c]);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t *>(&ws[t * 8 + g][kk + 2 * c + 8]);
-            mma_bf16_16816(acc[t], a[u], b0, b1);
-          }
-        }
-      }
-    }
-    __syncthreads();
-  }
-  float *dst = part + static_cast<int64_t>(blockIdx.y) * M * r;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int j = t * 8 + 2 * c;
-    if (va) {
-      if (j < r) dst[ra * r + j] = acc[t][0];
-      if (j + 1 < r) dst[ra * r + j + 1] = acc[t][1];
-    }
-    if (vb) {
-      if (j < r) dst[rb * r + j] = acc[t][2];
-      if (j + 1 < r) dst[rb * r + j + 1] = acc[t][3];
+__device__ __forceinline__ void producer_drain(uint64_t *full, uint32_t mask, uint32_t par) {
+  for (int s = 0; s < kStages; ++s) {
+    if (!(mask & (1u << s))) continue;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(&full[s], (par >> s) & 1u) && global_timer_ns() - t0 < kWaitLimitNs) {
     }
   }
 }
 
-__global__ void lora_rows_finalize(const float *__restrict__ part, int splits, int64_t n, float s,
-                                   uint16_t *__restrict__ out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float acc = 0.f;
-  for (int q = 0; q < splits; ++q) acc += part[q * n + i];
-  out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(s * acc));
-}
-
 // ---------------------------------------------------------------------------
-// cols: sum over m of Z[m, d] V[m, j] -> part[split][D][r] (fp32)
-// CTA = 8 warps over 128 columns (4 per lane) and 16 adapter columns (grid.z
-// picks the 16-wide slice of r); warps stride over the CTA's rows.
+// rows: 64 rows of Z per CTA (4 consumer warps x 16 rows) + 1 producer warp.
+// Stage = Z tile [64 m][64 k] (SW128) + adapter tile for the same 64 k:
+//   w_is_rk (W is [r, K]):  [r_pad j][64 k], SW128
+//   otherwise (W is [K, r]): [64 k][r_pad j], swizzle span 2 * r_pad
 // ---------------------------------------------------------------------------
-constexpr int kColsWarps = 8;
-constexpr int kColsD = 128;
-constexpr int kColsRowsMax = 256;   // rows per CTA (V slice staged in smem)
-
-__global__ void __launch_bounds__(32 * kColsWarps) lora_cols_ffma2(const uint16_t *__restrict__ Z, int64_t M,
-                                                                    int64_t D, const uint16_t *__restrict__ V,
-                                                                    int r, int64_t m_per_split,
-                                                                    float *__restrict__ part) {
-  extern __shared__ __align__(16) float smem_cols[];
-  float *vs = smem_cols;                          // [kColsRowsMax][16]
-  float *red = smem_cols + kColsRowsMax * 16;     // [kColsWarps][32 lanes][64]
+template <int NT>   // n-tiles of 8 adapter columns: r_pad = 8 * NT (16, 32 or 64)
+__global__ void __launch_bounds__(160) lora_rows_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                        const __grid_constant__ CUtensorMap tm_w, int64_t M,
+                                                        int64_t K, int r, int w_is_rk, int kb_per_cta, float s,
+                                                        uint16_t *__restrict__ out, int32_t *status) {
+  constexpr int r_pad = NT * 8;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t z_bytes = 64 * 128;
+  constexpr uint32_t w_bytes = r_pad * 128;   // 64 k x r_pad j x 2 B
+  constexpr uint32_t stage_bytes = z_bytes + ((w_bytes + 1023u) & ~1023u);
+  float *red = reinterpret_cast<float *>(base + kStages * stage_bytes);   // [64][r_pad]
+  uint64_t *full = reinterpret_cast<uint64_t *>(red + 64 * r_pad);
+  uint64_t *empty = full + kStages;
+  int *abort_flag_p = reinterpret_cast<int *>(empty + kStages);
+  volatile int *abort_flag = abort_flag_p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t d0 = static_cast<int64_t>(blockIdx.x) * kColsD + lane * 4;
-  const int j0 = blockIdx.z * 16;
-  const int64_t mbeg = static_cast<int64_t>(blockIdx.y) * m_per_split;
-  const int64_t mend = min(M, mbeg + m_per_split);
-  const int rows = static_cast<int>(mend - mbeg);
+  const uint32_t rank = cluster_ctarank();
+  const int csize = static_cast<int>(gridDim.y);
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int kb_begin = static_cast<int>(blockIdx.y) * kb_per_cta;
+  const int kb_total = static_cast<int>((K + 63) / 64);
+  const int kb_end = kb_begin + kb_per_cta < kb_total ? kb_begin + kb_per_cta : kb_total;
+  const int nsteps = kb_end > kb_begin ? kb_end - kb_begin : 0;
 
-#pragma unroll 4
-  for (int e = threadIdx.x; e < rows * 16; e += blockDim.x) {
-    const int i = e >> 4, j = e & 15;
-    vs[e] = (j0 + j < r) ? __uint_as_float(static_cast<uint32_t>(__ldg(V + (mbeg + i) * r + j0 + j)) << 16) : 0.f;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    *abort_flag_p = 0;
+    fence_mbarrier_init();
   }
   __syncthreads();
 
-  float2 acc[4][8];
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[q][j] = make_float2(0.f, 0.f);
-
-  const bool dok = d0 < D;   // D % 4 == 0, so a lane's 4 columns are all in or all out
-  constexpr int kU = 8;      // rows whose loads are in flight together per warp
-  for (int i0 = warp; i0 < rows; i0 += kU * kColsWarps) {
-    uint2 zw[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = i0 + u * kColsWarps;
-      zw[u] = (dok && i < rows) ? __ldg(reinterpret_cast<const uint2 *>(Z + (mbeg + i) * D + d0))
-                                : make_uint2(0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int i = i0 + u * kColsWarps;
-      if (i < rows) {
-        const float x[4] = {__uint_as_float(zw[u].x << 16), __uint_as_float(zw[u].x & 0xFFFF0000u),
-                            __uint_as_float(zw[u].y << 16), __uint_as_float(zw[u].y & 0xFFFF0000u)};
-        const float4 *vr = reinterpret_cast<const float4 *>(vs + i * 16);
-        float2 v[8];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float4 t = vr[h];
-          v[2 * h] = make_float2(t.x, t.y);
-          v[2 * h + 1] = make_float2(t.z, t.w);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 xx = make_float2(x[q], x[q]);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[q][j] = __ffma2_rn(xx, v[j], acc[q][j]);
-        }
+  if (warp == 4) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_z);
+      tma_prefetch_desc(&tm_w);
+      uint32_t mask = 0, par = 0;
+      int slot = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag, status)) break;
+        uint8_t *st = base + slot * stage_bytes;
+        mbar_arrive_expect_tx(&full[slot], z_bytes + w_bytes);
+        const int k0 = (kb_begin + i) * 64;
+        tma_load_2d(st, &tm_z, &full[slot], k0, static_cast<int32_t>(m0));
+        if (w_is_rk) tma_load_2d(st + z_bytes, &tm_w, &full[slot], k0, 0);
+        else         tma_load_2d(st + z_bytes, &tm_w, &full[slot], 0, k0);
+        mask |= 1u << slot;
+        par = (par & ~(1u << slot)) | (ph << slot);
+        if (++slot == kStages) { slot = 0; ph ^= 1u; }
       }
+      if (*abort_flag) producer_drain(full, mask, par);
     }
-  }
-  // reduce the 8 warps' accumulators in a fixed order
-  float *mine = red + (warp * 32 + lane) * 64;
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      mine[q * 16 + 2 * j] = acc[q][j].x;
-      mine[q * 16 + 2 * j + 1] = acc[q][j].y;
-    }
-  __syncthreads();
-  float *dst = part + static_cast<int64_t>(blockIdx.y) * D * r;
-  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
-    const int ln = e >> 6, qj = e & 63;
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kColsWarps; ++w) sum += red[(w * 32 + ln) * 64 + qj];
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * kColsD + ln * 4 + (qj >> 4);
-    const int j = j0 + (qj & 15);
-    if (d < D && j < r) dst[d * r + j] = sum;
-  }
-}
-
-__global__ void lora_cols_finalize(const float *__restrict__ part, int splits, int64_t D, int r,
-                                   int transpose_out, float *__restrict__ out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = D * r;
-  if (i >= n) return;
-  float acc = 0.f;
-  for (int q = 0; q < splits; ++q) acc += part[q * n + i];
-  if (transpose_out) {
-    const int64_t d = i / r, j = i % r;
-    out[j * D + d] = acc;
   } else {
-    out[i] = acc;
+    float acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    const uint32_t wspan = w_is_rk ? 128u : static_cast<uint32_t>(2 * r_pad);
+    int slot = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nsteps; ++i) {
+      if (!mbar_wait(&full[slot], ph, abort_flag, status)) break;
+      const uint32_t zs = smem_u32(base + slot * stage_bytes);
+      const uint32_t wsm = zs + z_bytes;
+#pragma unroll
+      for (int kk = 0; kk < 64; kk += 16) {
+        uint32_t a[4];
+        {
+          const uint32_t row = static_cast<uint32_t>(warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8);
+          const uint32_t chunk = static_cast<uint32_t>(kk / 8 + (lane >> 4));
+          ldmatrix_x4(a, zs + swizzle_off(row * 128u + chunk * 16u, kSpanZ));
+        }
+#pragma unroll
+        for (int t = 0; t < NT; t += 2) {
+          uint32_t b[4];
+          if (w_is_rk) {
+            // tile [j][k]: matrices (j-tile t, k chunk c), (t, c+1), (t+1, c), (t+1, c+1)
+            const uint32_t j = static_cast<uint32_t>(8 * (t + (lane >> 4)) + (lane & 7));
+            const uint32_t chunk = static_cast<uint32_t>(kk / 8 + ((lane >> 3) & 1));
+            ldmatrix_x4(b, wsm + swizzle_off(j * 128u + chunk * 16u, wspan));
+          } else {
+            // tile [k][j], transposed 8x8 loads: (k rows kk.., j-tile t), (kk+8.., t), (kk.., t+1), (kk+8.., t+1)
+            const uint32_t krow = static_cast<uint32_t>(kk + (lane & 7) + ((lane >> 3) & 1) * 8);
+            const uint32_t chunk = static_cast<uint32_t>(t + (lane >> 4));
+            ldmatrix_x4_trans(b, wsm + swizzle_off(krow * wspan + chunk * 16u, wspan));
+          }
+          mma_16816(acc[t], a, b[0], b[1]);
+          mma_16816(acc[t + 1], a, b[2], b[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (++slot == kStages) { slot = 0; ph ^= 1u; }
+    }
+    // this CTA's partial sums -> shared memory (row-major [64][r_pad])
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int row = warp * 16 + g, col = t * 8 + 2 * c;
+      red[row * r_pad + col] = acc[t][0];
+      red[row * r_pad + col + 1] = acc[t][1];
+      red[(row + 8) * r_pad + col] = acc[t][2];
+      red[(row + 8) * r_pad + col + 1] = acc[t][3];
+    }
   }
+  // add the cluster's partials in rank order: rank q owns rows [q*64/csize, ..)
+  cluster_sync_all();
+  const int rows_per = (64 + csize - 1) / csize;
+  const int r_lo = static_cast<int>(rank) * rows_per;
+  const int r_hi = r_lo + rows_per < 64 ? r_lo + rows_per : 64;
+  const uint32_t red_addr = smem_u32(red);
+  for (int e = threadIdx.x; e < (r_hi - r_lo) * r; e += blockDim.x) {
+    const int row = r_lo + e / r, j = e % r;
+    const int64_t m = m0 + row;
+    if (m >= M) continue;
+    const uint32_t off = static_cast<uint32_t>((row * r_pad + j) * 4);
+    float sum = 0.f;
+    for (int q = 0; q < csize; ++q) sum += ld_dsmem_f32(mapa_shared(red_addr + off, static_cast<uint32_t>(q)));
+    out[m * r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s * sum));
+  }
+  cluster_sync_all();
 }
 
-int rows_splits(int64_t M, int64_t K) {
-  const int64_t ctas = (M + kRowsTile - 1) / kRowsTile;
-  const int64_t chunks = (K + kKC - 1) / kKC;
-  int64_t s = (2 * device_sm_count() + ctas - 1) / ctas;
-  if (s > chunks) s = chunks;
-  if (s < 1) s = 1;
-  return static_cast<int>(s);
-}
-
-int cols_splits(int64_t M, int64_t D) {
-  const int64_t ctas = (D + kColsD - 1) / kColsD;
-  const int64_t chunks = (M + kColsRowsMax - 1) / kColsRowsMax;   // at most kColsRowsMax rows per CTA
-  int64_t s = (2 * device_sm_count() + ctas - 1) / ctas;
-  if (s < chunks) s = chunks;
-  const int64_t max_s = (M + 7) / 8;    // keep at least 8 rows per split
-  if (s > max_s) s = max_s;
-  if (s < chunks) s = chunks;
-  if (s < 1) s = 1;
-  return static_cast<int>(s);
-}
-
-size_t cols_smem_bytes() { return (kColsRowsMax * 16 + kColsWarps * 32 * 64) * sizeof(float); }
-
+// ---------------------------------------------------------------------------
+// cols: 128 columns of Z per CTA (8 consumer warps x 16 columns) + 1 producer
+// warp. Stage = Z tile [64 m][128 d] as two SW128 boxes of 64 columns, and the
+// V tile [64 m][r_pad j] (swizzle span 2 * r_pad).
+// ---------------------------------------------------------------------------
 template <int NT>
-cudaError_t rows_launch(dim3 grid, cudaStream_t st, const uint16_t *Z, int64_t M, int64_t K, const uint16_t *W,
-                        int r, bool w_is_rk, int64_t kps, float *ws) {
-  lora_rows_mma<NT><<<grid, 32 * kRowsWarps, 0, st>>>(Z, M, K, W, r, w_is_rk ? 1 : 0, kps, ws);
-  return cudaGetLastError();
+__global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                                        const __grid_constant__ CUtensorMap tm_v, int64_t M,
+                                                        int64_t D, int r, int mb_per_cta, int transpose_out,
+                                                        float *__restrict__ out, int32_t *status) {
+  constexpr int r_pad = NT * 8;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t z_bytes = 2 * 64 * 128;    // two boxes of [64 m][64 d]
+  constexpr uint32_t v_bytes = r_pad * 128;     // [64 m][r_pad] bf16
+  constexpr uint32_t stage_bytes = z_bytes + ((v_bytes + 1023u) & ~1023u);
+  constexpr uint32_t vspan = 2 * r_pad;
+  float *red = reinterpret_cast<float *>(base + kStages * stage_bytes);   // [128][r_pad]
+  uint64_t *full = reinterpret_cast<uint64_t *>(red + 128 * r_pad);
+  uint64_t *empty = full + kStages;
+  int *abort_flag_p = reinterpret_cast<int *>(empty + kStages);
+  volatile int *abort_flag = abort_flag_p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int csize = static_cast<int>(gridDim.y);
+  const int64_t d0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int mb_begin = static_cast<int>(blockIdx.y) * mb_per_cta;
+  const int mb_total = static_cast<int>((M + 63) / 64);
+  const int mb_end = mb_begin + mb_per_cta < mb_total ? mb_begin + mb_per_cta : mb_total;
+  const int nsteps = mb_end > mb_begin ? mb_end - mb_begin : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 8);
+    }
+    *abort_flag_p = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_z);
+      tma_prefetch_desc(&tm_v);
+      uint32_t mask = 0, par = 0;
+      int slot = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag, status)) break;
+        uint8_t *st = base + slot * stage_bytes;
+        mbar_arrive_expect_tx(&full[slot], z_bytes + v_bytes);
+        const int mrow = (mb_begin + i) * 64;
+        tma_load_2d(st, &tm_z, &full[slot], static_cast<int32_t>(d0), mrow);
+        tma_load_2d(st + 64 * 128, &tm_z, &full[slot], static_cast<int32_t>(d0 + 64), mrow);
+        tma_load_2d(st + z_bytes, &tm_v, &full[slot], 0, mrow);
+        mask |= 1u << slot;
+        par = (par & ~(1u << slot)) | (ph << slot);
+        if (++slot == kStages) { slot = 0; ph ^= 1u; }
+      }
+      if (*abort_flag) producer_drain(full, mask, par);
+    }
+  } else {
+    float acc[NT][4];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    // warp w: columns 16w..16w+15 = box w/4, 16-column group w%4 inside the box
+    const uint32_t box_off = static_cast<uint32_t>((warp >> 2) * 64 * 128);
+    const uint32_t dchunk0 = static_cast<uint32_t>((warp & 3) * 2);
+    int slot = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nsteps; ++i) {
+      if (!mbar_wait(&full[slot], ph, abort_flag, status)) break;
+      const uint32_t zs = smem_u32(base + slot * stage_bytes) + box_off;
+      const uint32_t vs = smem_u32(base + slot * stage_bytes) + z_bytes;
+#pragma unroll
+      for (int mm = 0; mm < 64; mm += 16) {
+        uint32_t a[4];   // Z^T fragment: rows = 16 columns d, cols = 16 rows m
+        {
+          const uint32_t mrow = static_cast<uint32_t>(mm + (lane & 7) + ((lane >> 4) & 1) * 8);
+          const uint32_t chunk = dchunk0 + static_cast<uint32_t>((lane >> 3) & 1);
+          ldmatrix_x4_trans(a, zs + swizzle_off(mrow * 128u + chunk * 16u, kSpanZ));
+        }
+#pragma unroll
+        for (int t = 0; t < NT; t += 2) {
+          uint32_t b[4];
+          const uint32_t mrow = static_cast<uint32_t>(mm + (lane & 7) + ((lane >> 3) & 1) * 8);
+          const uint32_t chunk = static_cast<uint32_t>(t + (lane >> 4));
+          ldmatrix_x4_trans(b, vs + swizzle_off(mrow * vspan + chunk * 16u, vspan));
+          mma_16816(acc[t], a, b[0], b[1]);
+          mma_16816(acc[t + 1], a, b[2], b[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (++slot == kStages) { slot = 0; ph ^= 1u; }
+    }
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int row = warp * 16 + g, col = t * 8 + 2 * c;
+      red[row * r_pad + col] = acc[t][0];
+      red[row * r_pad + col + 1] = acc[t][1];
+      red[(row + 8) * r_pad + col] = acc[t][2];
+      red[(row + 8) * r_pad + col + 1] = acc[t][3];
+    }
+  }
+  cluster_sync_all();
+  const int rows_per = (128 + csize - 1) / csize;
+  const int r_lo = static_cast<int>(rank) * rows_per;
+  const int r_hi = r_lo + rows_per < 128 ? r_lo + rows_per : 128;
+  const uint32_t red_addr = smem_u32(red);
+  for (int e = threadIdx.x; e < (r_hi - r_lo) * r; e += blockDim.x) {
+    const int row = r_lo + e / r, j = e % r;
+    const int64_t d = d0 + row;
+    if (d >= D) continue;
+    const uint32_t off = static_cast<uint32_t>((row * r_pad + j) * 4);
+    float sum = 0.f;
+    for (int q = 0; q < csize; ++q) sum += ld_dsmem_f32(mapa_shared(red_addr + off, static_cast<uint32_t>(q)));
+    if (transpose_out) out[static_cast<int64_t>(j) * D + d] = sum;
+    else               out[d * r + j] = sum;
+  }
+  cluster_sync_all();
+}
+
+int pad_rank(int r) { return r <= 16 ? 16 : (r <= 32 ? 32 : 64); }
+
+size_t rows_smem(int r_pad) {
+  const size_t stage = 64 * 128 + ((static_cast<size_t>(r_pad) * 128 + 1023) & ~size_t(1023));
+  return 1024 + kStages * stage + 64 * r_pad * 4 + 2 * kStages * 8 + 16;
+}
+size_t cols_smem(int r_pad) {
+  const size_t stage = 2 * 64 * 128 + ((static_cast<size_t>(r_pad) * 128 + 1023) & ~size_t(1023));
+  return 1024 + kStages * stage + 128 * r_pad * 4 + 2 * kStages * 8 + 16;
+}
+
+// Cluster size for splitting a reduction of `blocks` 64-wide steps when
+// `tiles` CTAs already cover the output: enough CTAs to fill the GPU twice.
+int cluster_split(int64_t tiles, int64_t blocks) {
+  int64_t c = (2 * device_sm_count() + tiles - 1) / tiles;
+  if (c > kClusterMax) c = kClusterMax;
+  if (c > blocks) c = blocks;
+  if (c < 1) c = 1;
+  return static_cast<int>(c);
+}
+
+template <typename Kernel>
+cudaError_t launch_cluster(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, int csize,
+                           void **args) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(csize);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(kernel), args);
 }
 
 }  // namespace
 
-size_t lora_rows_ws_floats(int64_t M, int64_t K, int r) {
-  return static_cast<size_t>(rows_splits(M, K)) * M * r;
-}
-size_t lora_cols_ws_floats(int64_t M, int64_t D, int r) {
-  return static_cast<size_t>(cols_splits(M, D)) * D * r;
-}
+// The skinny products keep their partial sums in shared memory: no workspace.
+size_t lora_rows_ws_floats(int64_t, int64_t, int) { return 0; }
+size_t lora_cols_ws_floats(int64_t, int64_t, int) { return 0; }
 
-cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint16_t *W, int r,
-                             bool w_is_rk, float s, uint16_t *out, float *ws, size_t ws_floats,
-                             cudaStream_t st) {
-  const int splits = rows_splits(M, K);
-  if (static_cast<size_t>(splits) * M * r > ws_floats) return cudaErrorInvalidValue;
-  const int64_t chunks = (K + kKC - 1) / kKC;
-  const int64_t k_per_split = ((chunks + splits - 1) / splits) * kKC;
-  const int real_splits = static_cast<int>((K + k_per_split - 1) / k_per_split);
-  dim3 grid(static_cast<unsigned>((M + kRowsTile - 1) / kRowsTile), static_cast<unsigned>(real_splits));
-  cudaError_t e;
-  switch ((r + 7) / 8) {
-    case 1: e = rows_launch<1>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 2: e = rows_launch<2>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 3: e = rows_launch<3>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 4: e = rows_launch<4>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 5: e = rows_launch<5>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 6: e = rows_launch<6>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 7: e = rows_launch<7>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
-    case 8: e = rows_launch<8>(grid, st, Z, M, K, W, r, w_is_rk, k_per_split, ws); break;
+cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint16_t *W, int r, bool w_is_rk,
+                             float s, uint16_t *out, float *, size_t, cudaStream_t st) {
+  const int r_pad = pad_rank(r);
+  CUtensorMap tm_z, tm_w;
+  bool ok = encode_2d(&tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Z, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (w_is_rk) ok &= encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, K, r, K * 2, 64, r_pad,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  else         ok &= encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, r, K, r * 2, r_pad, 64,
+                               swizzle_for_span(2 * r_pad));
+  if (!ok) return cudaErrorInvalidValue;
+  const int64_t mtiles = (M + 63) / 64;
+  const int64_t kblocks = (K + 63) / 64;
+  const int csize = cluster_split(mtiles, kblocks);
+  int kb_per_cta = static_cast<int>((kblocks + csize - 1) / csize);
+  int w_rk = w_is_rk ? 1 : 0;
+  int32_t *status = nullptr;
+  int64_t Mv = M, Kv = K;
+  int rv = r;
+  float sv = s;
+  void *args[] = {&tm_z, &tm_w, &Mv, &Kv, &rv, &w_rk, &kb_per_cta, &sv, &out, &status};
+  const dim3 grid(static_cast<unsigned>(mtiles), static_cast<unsigned>(csize));
+  const size_t smem = rows_smem(r_pad);
+  switch (r_pad / 8) {
+    case 2: return launch_cluster(lora_rows_kernel<2>, grid, 160, smem, st, csize, args);
+    case 4: return launch_cluster(lora_rows_kernel<4>, grid, 160, smem, st, csize, args);
+    case 8: return launch_cluster(lora_rows_kernel<8>, grid, 160, smem, st, csize, args);
     default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess) return e;
-  const int64_t n = M * r;
-  lora_rows_finalize<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(ws, real_splits, n, s, out);
-  return cudaGetLastError();
 }
 
-cudaError_t launch_lora_cols(const uint16_t *Z, int64_t M, int64_t D, const uint16_t *V, int r,
-                             bool transpose_out, float *out, float *ws, size_t ws_floats,
-                             cudaStream_t st) {
-  const int splits = cols_splits(M, D);
-  if (static_cast<size_t>(splits) * D * r > ws_floats) return cudaErrorInvalidValue;
-  const int64_t m_per_split = (M + splits - 1) / splits;
-  const int real_splits = static_cast<int>((M + m_per_split - 1) / m_per_split);
-  const size_t smem = cols_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(lora_cols_ffma2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>((D + kColsD - 1) / kColsD), static_cast<unsigned>(real_splits),
-            static_cast<unsigned>((r + 15) / 16));
-  lora_cols_ffma2<<<grid, 32 * kColsWarps, smem, st>>>(Z, M, D, V, r, m_per_split, ws);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int64_t n = D * r;
-  lora_cols_finalize<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(ws, real_splits, D, r,
-                                                                             transpose_out ? 1 : 0, out);
-  return cudaGetLastError();
+cudaError_t launch_lora_cols(const uint16_t *Z, int64_t M, int64_t D, const uint16_t *V, int r, bool transpose_out,
+                             float *out, float *, size_t, cudaStream_t st) {
+  const int r_pad = pad_rank(r);
+  CUtensorMap tm_z, tm_v;
+  bool ok = encode_2d(&tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Z, D, M, D * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_2d(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, r, M, r * 2, r_pad, 64, swizzle_for_span(2 * r_pad));
+  if (!ok) return cudaErrorInvalidValue;
+  const int64_t dtiles = (D + 127) / 128;
+  const int64_t mblocks = (M + 63) / 64;
+  const int csize = cluster_split(dtiles, mblocks);
+  int mb_per_cta = static_cast<int>((mblocks + csize - 1) / csize);
+  int tr = transpose_out ? 1 : 0;
+  int32_t *status = nullptr;
+  int64_t Mv = M, Dv = D;
+  int rv = r;
+  void *args[] = {&tm_z, &tm_v, &Mv, &Dv, &rv, &mb_per_cta, &tr, &out, &status};
+  const dim3 grid(static_cast<unsigned>(dtiles), static_cast<unsigned>(csize));
+  const size_t smem = cols_smem(r_pad);
+  switch (r_pad / 8) {
+    case 2: return launch_cluster(lora_cols_kernel<2>, grid, 288, smem, st, csize, args);
+    case 4: return launch_cluster(lora_cols_kernel<4>, grid, 288, smem, st, csize, args);
+    case 8: return launch_cluster(lora_cols_kernel<8>, grid, 288, smem, st, csize, args);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qlora
