@@ -226,12 +226,7 @@ qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M
   const size_t fa = lora_cols_ws_floats(M, K, r), fb = lora_cols_ws_floats(M, N, r);
   const size_t need = 4 * (fa > fb ? fa : fb);
   if (need > 0 && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  float *part = static_cast<float *>(ws);
-  // dA[j, k] = sum_m sT[m, j] X[m, k];  dB[n, j] = sum_m dY[m, n] sU[m, j]
-  cudaError_t e = launch_lora_cols(X, M, K, sT, r, /*transpose_out=*/true, dA, part, ws_bytes / 4, cs);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
-  return cuda_status(launch_lora_cols(dY, M, N, sU, r, /*transpose_out=*/false, dB, part, ws_bytes / 4, cs));
+  return cuda_status(launch_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,

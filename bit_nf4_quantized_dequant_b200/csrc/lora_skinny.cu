@@ -22,7 +22,8 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, ui
 
 namespace {
 
-constexpr int kStages = 6;
+constexpr int kStages = 6;       // rows ring depth
+constexpr int kStagesCols = 4;   // cols ring depth (two CTAs fit per SM)
 constexpr int kClusterMax = 8;
 constexpr uint32_t kSpanZ = 128;   // Z tiles: 64 bf16 per row, SWIZZLE_128B
 
@@ -175,13 +176,23 @@ __global__ void __launch_bounds__(160) lora_rows_kernel(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 // cols: 128 columns of Z per CTA (8 consumer warps x 16 columns) + 1 producer
 // warp. Stage = Z tile [64 m][128 d] as two SW128 boxes of 64 columns, and the
-// V tile [64 m][r_pad j] (swizzle span 2 * r_pad).
+// V tile [64 m][r_pad j] (swizzle span 2 * r_pad). One launch serves two
+// products (dA = sT^T X with transposed output, dB = dY^T sU): CTAs with
+// blockIdx.x < tiles0 take the first, the rest the second.
 // ---------------------------------------------------------------------------
+struct ColsProblem {
+  int64_t D;
+  float *out;
+  int transpose_out;
+};
+
 template <int NT>
-__global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ CUtensorMap tm_z,
-                                                        const __grid_constant__ CUtensorMap tm_v, int64_t M,
-                                                        int64_t D, int r, int mb_per_cta, int transpose_out,
-                                                        float *__restrict__ out, int32_t *status) {
+__global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ CUtensorMap tm_z0,
+                                                        const __grid_constant__ CUtensorMap tm_v0,
+                                                        const __grid_constant__ CUtensorMap tm_z1,
+                                                        const __grid_constant__ CUtensorMap tm_v1, ColsProblem p0,
+                                                        ColsProblem p1, int tiles0, int64_t M, int r,
+                                                        int mb_per_cta, int32_t *status) {
   constexpr int r_pad = NT * 8;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -189,22 +200,26 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
   constexpr uint32_t v_bytes = r_pad * 128;     // [64 m][r_pad] bf16
   constexpr uint32_t stage_bytes = z_bytes + ((v_bytes + 1023u) & ~1023u);
   constexpr uint32_t vspan = 2 * r_pad;
-  float *red = reinterpret_cast<float *>(base + kStages * stage_bytes);   // [128][r_pad]
+  float *red = reinterpret_cast<float *>(base + kStagesCols * stage_bytes);   // [128][r_pad]
   uint64_t *full = reinterpret_cast<uint64_t *>(red + 128 * r_pad);
-  uint64_t *empty = full + kStages;
-  int *abort_flag_p = reinterpret_cast<int *>(empty + kStages);
+  uint64_t *empty = full + kStagesCols;
+  int *abort_flag_p = reinterpret_cast<int *>(empty + kStagesCols);
   volatile int *abort_flag = abort_flag_p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int csize = static_cast<int>(gridDim.y);
-  const int64_t d0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const bool second = static_cast<int>(blockIdx.x) >= tiles0;
+  const CUtensorMap *tm_z = second ? &tm_z1 : &tm_z0;
+  const CUtensorMap *tm_v = second ? &tm_v1 : &tm_v0;
+  const ColsProblem pr = second ? p1 : p0;
+  const int64_t d0 = static_cast<int64_t>(second ? static_cast<int>(blockIdx.x) - tiles0 : static_cast<int>(blockIdx.x)) * 128;
   const int mb_begin = static_cast<int>(blockIdx.y) * mb_per_cta;
   const int mb_total = static_cast<int>((M + 63) / 64);
   const int mb_end = mb_begin + mb_per_cta < mb_total ? mb_begin + mb_per_cta : mb_total;
   const int nsteps = mb_end > mb_begin ? mb_end - mb_begin : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kStagesCols; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 8);
     }
@@ -215,8 +230,8 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
 
   if (warp == 8) {
     if (elect_one()) {
-      tma_prefetch_desc(&tm_z);
-      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(tm_z);
+      tma_prefetch_desc(tm_v);
       uint32_t mask = 0, par = 0;
       int slot = 0;
       uint32_t ph = 0;
@@ -225,14 +240,21 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
         uint8_t *st = base + slot * stage_bytes;
         mbar_arrive_expect_tx(&full[slot], z_bytes + v_bytes);
         const int mrow = (mb_begin + i) * 64;
-        tma_load_2d(st, &tm_z, &full[slot], static_cast<int32_t>(d0), mrow);
-        tma_load_2d(st + 64 * 128, &tm_z, &full[slot], static_cast<int32_t>(d0 + 64), mrow);
-        tma_load_2d(st + z_bytes, &tm_v, &full[slot], 0, mrow);
+        tma_load_2d(st, tm_z, &full[slot], static_cast<int32_t>(d0), mrow);
+        tma_load_2d(st + 64 * 128, tm_z, &full[slot], static_cast<int32_t>(d0 + 64), mrow);
+        tma_load_2d(st + z_bytes, tm_v, &full[slot], 0, mrow);
         mask |= 1u << slot;
         par = (par & ~(1u << slot)) | (ph << slot);
-        if (++slot == kStages) { slot = 0; ph ^= 1u; }
+        if (++slot == kStagesCols) { slot = 0; ph ^= 1u; }
       }
-      if (*abort_flag) producer_drain(full, mask, par);
+      if (*abort_flag) {
+        for (int q = 0; q < kStagesCols; ++q) {
+          if (!(mask & (1u << q))) continue;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[q], (par >> q) & 1u) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
     }
   } else {
     float acc[NT][4];
@@ -267,7 +289,7 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
-      if (++slot == kStages) { slot = 0; ph ^= 1u; }
+      if (++slot == kStagesCols) { slot = 0; ph ^= 1u; }
     }
     const int g = lane >> 2, c = lane & 3;
 #pragma unroll
@@ -287,12 +309,12 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
   for (int e = threadIdx.x; e < (r_hi - r_lo) * r; e += blockDim.x) {
     const int row = r_lo + e / r, j = e % r;
     const int64_t d = d0 + row;
-    if (d >= D) continue;
+    if (d >= pr.D) continue;
     const uint32_t off = static_cast<uint32_t>((row * r_pad + j) * 4);
     float sum = 0.f;
     for (int q = 0; q < csize; ++q) sum += ld_dsmem_f32(mapa_shared(red_addr + off, static_cast<uint32_t>(q)));
-    if (transpose_out) out[static_cast<int64_t>(j) * D + d] = sum;
-    else               out[d * r + j] = sum;
+    if (pr.transpose_out) pr.out[static_cast<int64_t>(j) * pr.D + d] = sum;
+    else                  pr.out[d * r + j] = sum;
   }
   cluster_sync_all();
 }
@@ -305,7 +327,7 @@ size_t rows_smem(int r_pad) {
 }
 size_t cols_smem(int r_pad) {
   const size_t stage = 2 * 64 * 128 + ((static_cast<size_t>(r_pad) * 128 + 1023) & ~size_t(1023));
-  return 1024 + kStages * stage + 128 * r_pad * 4 + 2 * kStages * 8 + 16;
+  return 1024 + kStagesCols * stage + 128 * r_pad * 4 + 2 * kStagesCols * 8 + 16;
 }
 
 // Cluster size for splitting a reduction of `blocks` 64-wide steps when
@@ -374,23 +396,29 @@ cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint
   }
 }
 
-cudaError_t launch_lora_cols(const uint16_t *Z, int64_t M, int64_t D, const uint16_t *V, int r, bool transpose_out,
-                             float *out, float *, size_t, cudaStream_t st) {
+cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st) {
   const int r_pad = pad_rank(r);
-  CUtensorMap tm_z, tm_v;
-  bool ok = encode_2d(&tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Z, D, M, D * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= encode_2d(&tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, r, M, r * 2, r_pad, 64, swizzle_for_span(2 * r_pad));
+  CUtensorMap tz0, tv0, tz1, tv1;
+  // product 0: dA[j, k] = sum_m sT[m, j] X[m, k]  (D = K, transposed output)
+  // product 1: dB[n, j] = sum_m dY[m, n] sU[m, j] (D = N)
+  bool ok = encode_2d(&tz0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_2d(&tv0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sT, r, M, r * 2, r_pad, 64, swizzle_for_span(2 * r_pad));
+  ok &= encode_2d(&tz1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= encode_2d(&tv1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sU, r, M, r * 2, r_pad, 64, swizzle_for_span(2 * r_pad));
   if (!ok) return cudaErrorInvalidValue;
-  const int64_t dtiles = (D + 127) / 128;
+  const int tiles0 = static_cast<int>((K + 127) / 128);
+  const int tiles1 = static_cast<int>((N + 127) / 128);
   const int64_t mblocks = (M + 63) / 64;
-  const int csize = cluster_split(dtiles, mblocks);
+  const int csize = cluster_split(tiles0 + tiles1, mblocks);
   int mb_per_cta = static_cast<int>((mblocks + csize - 1) / csize);
-  int tr = transpose_out ? 1 : 0;
-  int32_t *status = nullptr;
-  int64_t Mv = M, Dv = D;
+  ColsProblem p0{K, dA, 1}, p1{N, dB, 0};
+  int t0v = tiles0;
+  int64_t Mv = M;
   int rv = r;
-  void *args[] = {&tm_z, &tm_v, &Mv, &Dv, &rv, &mb_per_cta, &tr, &out, &status};
-  const dim3 grid(static_cast<unsigned>(dtiles), static_cast<unsigned>(csize));
+  int32_t *status = nullptr;
+  void *args[] = {&tz0, &tv0, &tz1, &tv1, &p0, &p1, &t0v, &Mv, &rv, &mb_per_cta, &status};
+  const dim3 grid(static_cast<unsigned>(tiles0 + tiles1), static_cast<unsigned>(csize));
   const size_t smem = cols_smem(r_pad);
   switch (r_pad / 8) {
     case 2: return launch_cluster(lora_cols_kernel<2>, grid, 288, smem, st, csize, args);

@@ -85,24 +85,41 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
 }
 
 // One thread per half block (32 weights = 16 code bytes -> 64 output bytes).
+// Each warp stages its 32 x 64 contiguous output bytes in shared memory and
+// writes them with one bulk copy, so global stores are full, contiguous 2 KiB
+// runs instead of 64-byte pieces strided across the warp.
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
                                                           const uint8_t *__restrict__ scale8,
                                                           const float *__restrict__ scale2,
                                                           int64_t nhalf, uint16_t *__restrict__ out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= nhalf) return;
-  const int64_t b = i >> 1;
-  const uint4 c = __ldg(reinterpret_cast<const uint4 *>(codes) + i);
-  const float sc = block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
-  const Nf4Table t = make_table(sc);
-  uint4 *dst = reinterpret_cast<uint4 *>(out) + i * 4;
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  __shared__ __align__(128) uint4 stage[8][32 * 4];   // per warp: 32 threads x 64 bytes
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t warp_first = (static_cast<int64_t>(blockIdx.x) * blockDim.x) + warp * 32;
+  if (warp_first >= nhalf) return;
+  const int64_t i = warp_first + lane;
+  const int active = static_cast<int>(nhalf - warp_first < 32 ? nhalf - warp_first : 32);
+  uint4 *mine = &stage[warp][lane * 4];
+  if (i < nhalf) {
+    const int64_t b = i >> 1;
+    const uint4 c = __ldg(reinterpret_cast<const uint4 *>(codes) + i);
+    const float sc = block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
+    const Nf4Table t = make_table(sc);
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t o[4];
-    expand8(t, w[q], o);
-    dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int k = 0; k < 4; ++k) {
+      uint32_t o[4];
+      expand8(t, w[k], o);
+      mine[k] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    bulk_store(out + warp_first * 32, &stage[warp][0], static_cast<uint32_t>(active) * 64u);
+    bulk_commit_group();
+    bulk_wait_group_read<0>();
+  }
+  __syncwarp();
 }
 
 }  // namespace

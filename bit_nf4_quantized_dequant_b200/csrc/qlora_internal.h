@@ -39,11 +39,10 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint16_t *W, int r,
                              bool w_is_rk, float s, uint16_t *out, float *ws, size_t ws_floats,
                              cudaStream_t st);
-// sum over m of Z[m, d] * V[m, j]  ->  out[d*r + j] (transpose_out = false) or
-// out[j*D + d] (transpose_out = true), fp32.
-cudaError_t launch_lora_cols(const uint16_t *Z, int64_t M, int64_t D, const uint16_t *V, int r,
-                             bool transpose_out, float *out, float *ws, size_t ws_floats,
-                             cudaStream_t st);
+// Adapter gradients in one launch: dA[j, k] = sum_m sT[m, j] X[m, k] and
+// dB[n, j] = sum_m dY[m, n] sU[m, j] (fp32, overwritten).
+cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st);
 size_t lora_rows_ws_floats(int64_t M, int64_t K, int r);
 size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
 
