@@ -7,8 +7,8 @@
 // activation gradient dX = dY W' + (alpha / r) (dY B) A but never dW.
 //
 // Both products are run "swap-AB": the dequantised weight tile is the UMMA A
-// operand (M = 128 weight rows or columns), the tokens are the UMMA N dimension
-// (BT up to 256), so each dequantised tile feeds 2 * 128 * BT flops.
+// operand (weight rows for FWD, weight columns for DX), the tokens are the UMMA
+// N dimension (BT up to 256), so each dequantised weight feeds 2 * BT flops.
 //
 //   FWD: D[n, t] = sum_k W'[n, k] X[t, k]  + sum_j Bl[n, j] sU[t, j]  -> Y[t, n]
 //        A tile K-major (W' rows are contiguous along k).
@@ -24,6 +24,14 @@
 // Two groups of four warps dequantise alternate K-steps, one thread per
 // 64-weight block.
 //
+// Two variants share this source. Single CTA: UMMA M = 128, one CTA per tile.
+// CTA pair (cta_group::2, a cluster of two): UMMA M = 256 across the pair; each
+// CTA dequantises its own 128 weight rows and loads half of the token tile, and
+// the pair's tensor cores read both halves, so every SM moves about a third
+// less data through shared memory per flop. The even CTA issues the MMAs; the
+// odd CTA's producers and dequantisers signal the even CTA's barriers, and the
+// even CTA's MMA completions are multicast to both.
+//
 // Warp roles (512 threads): 0 codes producer, 1 MMA issuer and TMEM owner,
 // 2 activation producer, 3 LoRA-slice producer, 4-7 epilogue (TMEM lane
 // quadrant = warp % 4; results leave through shared memory and TMA stores),
@@ -36,7 +44,7 @@ namespace qlora {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kTileRows = 128;                                // UMMA M
+constexpr int kTileRows = 128;                                // weight rows per CTA
 constexpr int kKStage = 64;                                   // K per step (one NF4 block)
 constexpr uint32_t kATileBytes = kTileRows * kKStage * 2;     // 16 KiB
 constexpr uint32_t kCodeTileBytes = kTileRows * kKStage / 2;  // 4 KiB
@@ -49,17 +57,18 @@ struct GemmParams {
   int32_t *status;
   int64_t N, K, M;
   int mode;        // 0 FWD, 1 DX
-  int bt;          // token tile (UMMA N)
+  int bt;          // token tile of one (pair) tile = UMMA N
+  int bt_cta;      // tokens whose activations this CTA loads (bt, or bt / 2 for a pair)
   int sx, sa, sc;  // ring depths: activations, dequantised tiles, codes
   int r_pad;       // LoRA K extent in smem (16, 32 or 64)
-  int row_tiles;   // tiles along the UMMA M dimension
+  int row_tiles;   // tiles along the weight dimension (128 rows, or 256 for a pair)
   int tok_tiles;
   int nk;          // main-loop K steps per tile
 };
 
 __host__ __device__ inline uint32_t lora_a_bytes(int r_pad) { return kTileRows * r_pad * 2; }
-__host__ __device__ inline uint32_t lora_b_bytes(int bt, int r_pad) {
-  return ((static_cast<uint32_t>(bt) * r_pad * 2 + 1023u) / 1024u) * 1024u;
+__host__ __device__ inline uint32_t lora_b_bytes(int bt_cta, int r_pad) {
+  return ((static_cast<uint32_t>(bt_cta) * r_pad * 2 + 1023u) / 1024u) * 1024u;
 }
 
 __device__ __forceinline__ uint32_t lora_layout(int r_pad) {
@@ -76,11 +85,11 @@ struct Smem {
 
 __device__ __forceinline__ Smem carve(uint8_t *base, const GemmParams &p) {
   Smem s;
-  s.x_bytes = static_cast<uint32_t>(p.bt) * 128u;
+  s.x_bytes = static_cast<uint32_t>(p.bt_cta) * 128u;
   uint8_t *ptr = base;
   s.x = ptr;   ptr += static_cast<size_t>(p.sx) * s.x_bytes;
   s.a = ptr;   ptr += static_cast<size_t>(p.sa) * kATileBytes;
-  s.lb = ptr;  ptr += lora_b_bytes(p.bt, p.r_pad);
+  s.lb = ptr;  ptr += lora_b_bytes(p.bt_cta, p.r_pad);
   s.la = ptr;  ptr += lora_a_bytes(p.r_pad);
   s.out = ptr; ptr += 2 * kOutStageBytes;
   s.c = ptr;   ptr += static_cast<size_t>(p.sc) * kCodeTileBytes;
@@ -109,37 +118,36 @@ struct RingPos {
   }
 };
 
+// Which tiles a CTA (or CTA pair) walks: tile = first + lt * stride.
+struct TileWalk {
+  int first, stride, row_tiles;
+};
+
 // (local tile, k-step) of a position in this CTA's step sequence, advanced
-// without division; rt is the tile's index along the UMMA M dimension.
+// without division; rt / tt are the tile's indices along weights / tokens.
 struct StepPos {
   int lt, k, rt, tt;
-  __device__ __forceinline__ void set_tile(int row_tiles) {
-    const int tile = static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x);
-    rt = tile % row_tiles;
-    tt = tile / row_tiles;
+  __device__ __forceinline__ void set_tile(const TileWalk &w) {
+    const int tile = w.first + lt * w.stride;
+    rt = tile % w.row_tiles;
+    tt = tile / w.row_tiles;
   }
-  __device__ __forceinline__ void init(int it, int nk, int row_tiles) {
+  __device__ __forceinline__ void init(int it, int nk, const TileWalk &w) {
     lt = it / nk;
     k = it - lt * nk;
-    set_tile(row_tiles);
+    set_tile(w);
   }
-  __device__ __forceinline__ void advance(int by, int nk, int row_tiles) {
+  __device__ __forceinline__ void advance(int by, int nk, const TileWalk &w) {
     k += by;
     if (k >= nk) {
       while (k >= nk) {
         k -= nk;
         ++lt;
       }
-      set_tile(row_tiles);
+      set_tile(w);
     }
   }
 };
-
-// Number of tiles this CTA processes (tiles blockIdx.x, blockIdx.x + gridDim.x, ...).
-__device__ __forceinline__ int local_tiles(int ntiles) {
-  const int b = static_cast<int>(blockIdx.x), g = static_cast<int>(gridDim.x);
-  return ntiles > b ? (ntiles - b + g - 1) / g : 0;
-}
 
 // On an abort, wait (bounded) until the copies this thread issued into a ring
 // have landed, so that no TMA write outlives the CTA's shared memory.
@@ -153,6 +161,7 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int slots, uint32_t i
   }
 }
 
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                           const __grid_constant__ CUtensorMap tm_codes,
@@ -165,20 +174,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool dx = p.mode == 1;
+  // CTA pair: rank 0 (even CTA) issues the MMAs; rank 1 is its peer.
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const TileWalk walk{kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x),
+                      kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x), p.row_tiles};
   const int ntiles = p.row_tiles * p.tok_tiles;
-  const int nlt = local_tiles(ntiles);
+  const int nlt = ntiles > walk.first ? (ntiles - walk.first + walk.stride - 1) / walk.stride : 0;
   const int total_steps = nlt * p.nk;
+  const int rows_per_tile = kPair ? 2 * kTileRows : kTileRows;
+  const int row_off = static_cast<int>(rank) * kTileRows;     // this CTA's weight rows inside the tile
+  const int tok_off = static_cast<int>(rank) * p.bt_cta;      // this CTA's tokens inside the tile
   // two accumulators of bt columns; at least 64 so a 32-column load of buffer 1 stays inside
   const uint32_t tmem_cols = static_cast<uint32_t>(2 * p.bt) < 64u ? 64u : static_cast<uint32_t>(2 * p.bt);
   volatile int *abort_flag = sm.abort_flag;
 
   if (threadIdx.x == 0) {
+    const uint32_t per_step = kPair ? 8u : 4u;   // dequantiser / epilogue warps that arrive, pair-wide
     for (int i = 0; i < p.sx; ++i) { mbar_init(&sm.xf[i], 1); mbar_init(&sm.xe[i], 1); }
-    for (int i = 0; i < p.sa; ++i) { mbar_init(&sm.af[i], 4); mbar_init(&sm.ae[i], 1); }
+    for (int i = 0; i < p.sa; ++i) { mbar_init(&sm.af[i], per_step); mbar_init(&sm.ae[i], 1); }
     for (int i = 0; i < p.sc; ++i) { mbar_init(&sm.cf[i], 1); mbar_init(&sm.ce[i], 4); }
     mbar_init(sm.lf, 1);
     mbar_init(sm.le, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&sm.accf[i], 1); mbar_init(&sm.acce[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&sm.accf[i], 1); mbar_init(&sm.acce[i], per_step); }
     mbar_init(sm.drain, 1);
     *sm.abort_flag = 0;
     fence_mbarrier_init();
@@ -191,86 +209,122 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
-    tmem_alloc(sm.tmem_holder, tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(sm.tmem_holder, tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(sm.tmem_holder, tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync_all();   // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem_holder;
   const int kb_row = static_cast<int>(p.K / kBlock);   // NF4 blocks per weight row
-  const int grid = static_cast<int>(gridDim.x);
+
+  // An mbarrier of the even CTA (this CTA's own when not paired).
+  auto leader_bar = [&](uint64_t *bar) -> uint32_t {
+    return kPair ? mapa_shared(smem_u32(bar), 0u) : smem_u32(bar);
+  };
+  auto arrive_leader = [&](uint64_t *bar) {
+    if constexpr (kPair) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0u));
+    else mbar_arrive(bar);
+  };
+  auto load_for_leader = [&](void *dst, const CUtensorMap *map, uint64_t *bar, int32_t x, int32_t y) {
+    if constexpr (kPair) tma_load_2d_pair(dst, map, leader_bar(bar), x, y);
+    else tma_load_2d(dst, map, bar, x, y);
+  };
 
   if (warp == 0) {
-    // ---------------- codes producer ----------------
+    // ---------------- codes producer (this CTA's weight rows only) ----------------
     if (elect_one()) {
       uint32_t mask = 0, par = 0;
       bool ok = true;
       RingPos c{0, 0};
       StepPos sp;
-      sp.init(0, p.nk, p.row_tiles);
-      for (int it = 0; it < total_steps; ++it, c.advance(1, p.sc), sp.advance(1, p.nk, p.row_tiles)) {
+      sp.init(0, p.nk, walk);
+      for (int it = 0; it < total_steps; ++it, c.advance(1, p.sc), sp.advance(1, p.nk, walk)) {
         const int s = c.slot;
         const uint32_t ph = c.phase;
         if (!mbar_wait(&sm.ce[s], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
         mbar_arrive_expect_tx(&sm.cf[s], kCodeTileBytes);
         uint8_t *cp = sm.c + static_cast<size_t>(s) * kCodeTileBytes;
-        if (!dx) tma_load_2d(cp, &tm_codes, &sm.cf[s], sp.k * (kKStage / 2), sp.rt * kTileRows);
-        else     tma_load_2d(cp, &tm_codes, &sm.cf[s], sp.rt * (kTileRows / 2), sp.k * kKStage);
+        const int r0 = sp.rt * rows_per_tile + row_off;
+        if (!dx) tma_load_2d(cp, &tm_codes, &sm.cf[s], sp.k * (kKStage / 2), r0);
+        else     tma_load_2d(cp, &tm_codes, &sm.cf[s], r0 / 2, sp.k * kKStage);
         mask |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       }
       if (!ok) drain_ring(sm.cf, p.sc, mask, par);
     }
   } else if (warp == 2) {
-    // ---------------- activation producer ----------------
+    // ---------------- activation producer (this CTA's tokens) ----------------
     if (elect_one()) {
       uint32_t mask = 0, par = 0;
       bool ok = true;
       RingPos x{0, 0};
       StepPos sp;
-      sp.init(0, p.nk, p.row_tiles);
-      for (int it = 0; it < total_steps; ++it, x.advance(1, p.sx), sp.advance(1, p.nk, p.row_tiles)) {
+      sp.init(0, p.nk, walk);
+      for (int it = 0; it < total_steps; ++it, x.advance(1, p.sx), sp.advance(1, p.nk, walk)) {
         const int s = x.slot;
         const uint32_t ph = x.phase;
         if (!mbar_wait(&sm.xe[s], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&sm.xf[s], sm.x_bytes);
-        tma_load_2d(sm.x + static_cast<size_t>(s) * sm.x_bytes, &tm_act, &sm.xf[s], sp.k * kKStage, sp.tt * p.bt);
+        if (leader) mbar_arrive_expect_tx(&sm.xf[s], kPair ? 2 * sm.x_bytes : sm.x_bytes);
+        load_for_leader(sm.x + static_cast<size_t>(s) * sm.x_bytes, &tm_act, &sm.xf[s], sp.k * kKStage,
+                        sp.tt * p.bt + tok_off);
         mask |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       }
-      if (!ok) drain_ring(sm.xf, p.sx, mask, par);
+      if (!ok && leader) drain_ring(sm.xf, p.sx, mask, par);
     }
   } else if (warp == 3) {
     // ---------------- LoRA-slice producer ----------------
     if (elect_one()) {
       bool issued = false;
       uint32_t last_ph = 0;
+      const uint32_t bytes_cta = lora_a_bytes(p.r_pad) + static_cast<uint32_t>(p.bt_cta) * p.r_pad * 2u;
       for (int lt = 0; lt < nlt; ++lt) {
-        const int tile = static_cast<int>(blockIdx.x) + lt * grid;
+        const int tile = walk.first + lt * walk.stride;
         const int rt = tile % p.row_tiles, tt = tile / p.row_tiles;
+        const int r0 = rt * rows_per_tile + row_off;
         const uint32_t ph = static_cast<uint32_t>(lt) & 1u;
         if (!mbar_wait(sm.le, ph ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(sm.lf, lora_a_bytes(p.r_pad) + static_cast<uint32_t>(p.bt) * p.r_pad * 2u);
-        tma_load_2d(sm.lb, &tm_lora_act, sm.lf, 0, tt * p.bt);
+        if (leader) mbar_arrive_expect_tx(sm.lf, kPair ? 2 * bytes_cta : bytes_cta);
+        load_for_leader(sm.lb, &tm_lora_act, sm.lf, 0, tt * p.bt + tok_off);
         if (!dx) {
-          tma_load_2d(sm.la, &tm_lora_w, sm.lf, 0, rt * kTileRows);
+          load_for_leader(sm.la, &tm_lora_w, sm.lf, 0, r0);
         } else {
-          tma_load_2d(sm.la, &tm_lora_w, sm.lf, rt * kTileRows, 0);
-          tma_load_2d(sm.la + p.r_pad * 128, &tm_lora_w, sm.lf, rt * kTileRows + 64, 0);
+          load_for_leader(sm.la, &tm_lora_w, sm.lf, r0, 0);
+          load_for_leader(sm.la + p.r_pad * 128, &tm_lora_w, sm.lf, r0 + 64, 0);
         }
         issued = true;
         last_ph = ph;
       }
-      if (*abort_flag && issued) drain_ring(sm.lf, 1, 1u, last_ph);
+      if (*abort_flag && issued && leader) drain_ring(sm.lf, 1, 1u, last_ph);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (elect_one()) {
-      const uint32_t idesc = idesc_bf16(kTileRows, static_cast<uint32_t>(p.bt), dx, false);
+    // ---------------- MMA issuer (the even CTA of a pair) ----------------
+    if (leader && elect_one()) {
+      const uint32_t idesc =
+          idesc_bf16(static_cast<uint32_t>(rows_per_tile), static_cast<uint32_t>(p.bt), dx, false);
       const uint32_t lsw = lora_layout(p.r_pad);
       const uint32_t lsbo = 16u * static_cast<uint32_t>(p.r_pad);   // 8 rows of 2 r_pad bytes
       const uint32_t la_addr = smem_u32(sm.la), lb_addr = smem_u32(sm.lb);
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t acc) {
+        if constexpr (kPair) umma_bf16_pair(d, ad, bd, idesc, acc);
+        else umma_bf16(d, ad, bd, idesc, acc);
+      };
+      auto commit = [&](uint64_t *bar) {
+        if constexpr (kPair) umma_commit_pair(bar);
+        else umma_commit(bar);
+      };
+      // K-step j of a slot: +32 bytes along K (K-major A) or +2 K-groups of 8 rows (MN-major A)
+      const uint64_t a_desc0 = dx ? smem_desc(smem_u32(sm.a), 8192u, 1024u, kLayoutSW128)
+                                  : smem_desc(smem_u32(sm.a), 16u, 1024u, kLayoutSW128);
+      const uint64_t b_desc0 = smem_desc(smem_u32(sm.x), 16u, 1024u, kLayoutSW128);
+      const uint32_t a_step = dx ? 2048u / 16u : 32u / 16u;
       bool ok = true, issued_any = false;
       RingPos xr{0, 0}, ar{0, 0};
       for (int lt = 0; lt < nlt && ok; ++lt) {
@@ -289,18 +343,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sm.a + static_cast<size_t>(as) * kATileBytes);
-          const uint32_t b_addr = smem_u32(sm.x + static_cast<size_t>(xs) * sm.x_bytes);
+          // descriptors = slot-0 descriptors + (byte offset >> 4) in the start-address field
+          const uint64_t a0 = a_desc0 + static_cast<uint64_t>((static_cast<uint32_t>(as) * kATileBytes) >> 4);
+          const uint64_t b0 = b_desc0 + static_cast<uint64_t>((static_cast<uint32_t>(xs) * sm.x_bytes) >> 4);
 #pragma unroll
           for (int j = 0; j < kKStage / 16; ++j) {
-            const uint64_t ad = dx ? smem_desc(a_addr + 2048u * j, 8192u, 1024u, kLayoutSW128)
-                                   : smem_desc(a_addr + 32u * j, 16u, 1024u, kLayoutSW128);
-            const uint64_t bd = smem_desc(b_addr + 32u * j, 16u, 1024u, kLayoutSW128);
-            umma_bf16(d_tmem, ad, bd, idesc, (k | j) != 0);
+            mma(d_tmem, a0 + static_cast<uint64_t>(a_step * j), b0 + static_cast<uint64_t>(2 * j), (k | j) != 0);
           }
           issued_any = true;
-          umma_commit(&sm.xe[xs]);
-          umma_commit(&sm.ae[as]);
+          commit(&sm.xe[xs]);
+          commit(&sm.ae[as]);
         }
         if (!ok) break;
         // LoRA K-steps: [.. | B] x [.. | sU] (FWD) or [.. ; A] x [.. | sT] (DX)
@@ -310,14 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = dx ? smem_desc(la_addr + 2048u * j, 128u * p.r_pad, 1024u, kLayoutSW128)
                                  : smem_desc(la_addr + 32u * j, 16u, lsbo, lsw);
           const uint64_t bd = smem_desc(lb_addr + 32u * j, 16u, lsbo, lsw);
-          umma_bf16(d_tmem, ad, bd, idesc, 1u);
+          mma(d_tmem, ad, bd, 1u);
         }
-        umma_commit(sm.le);
-        umma_commit(&sm.accf[buf]);
+        commit(sm.le);
+        commit(&sm.accf[buf]);
       }
       if (!ok && issued_any) {
         // drain: wait until every MMA issued so far has finished reading/writing
-        umma_commit(sm.drain);
+        commit(sm.drain);
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(sm.drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
@@ -326,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // ---------------- epilogue: TMEM -> bf16 -> smem -> TMA store ----------------
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
-    const int et = threadIdx.x - 128;       // 0..127 = row inside the tile
+    const int et = threadIdx.x - 128;       // 0..127 = this CTA's weight row inside the tile
     const int box_t = p.bt < kEpiTokens ? p.bt : kEpiTokens;
     const int nchunks = p.bt / box_t;
     uint32_t chunk_count = 0;
     for (int lt = 0; lt < nlt; ++lt) {
-      const int tile = static_cast<int>(blockIdx.x) + lt * grid;
+      const int tile = walk.first + lt * walk.stride;
       const int rt = tile % p.row_tiles, tt = tile / p.row_tiles;
       const int buf = lt & 1;
       if (!mbar_wait(&sm.accf[buf], static_cast<uint32_t>(lt >> 1) & 1u, abort_flag, p.status)) break;
@@ -345,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c == nchunks - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.acce[buf]);
+          if (lane == 0) arrive_leader(&sm.acce[buf]);
         }
         uint16_t *stage = reinterpret_cast<uint16_t *>(sm.out + (chunk_count & 1u) * kOutStageBytes);
         if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
@@ -358,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_barrier(1, 128);
         if (et == 0) {
-          tma_store_2d(&tm_out, stage, rt * kTileRows, tt * p.bt + c * box_t);
+          tma_store_2d(&tm_out, stage, rt * rows_per_tile + row_off, tt * p.bt + c * box_t);
           bulk_commit_group();
         }
       }
@@ -383,8 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       d = 0.f;
       if (it >= total_steps) return;
       int64_t n, kb;
-      if (!dx) { n = static_cast<int64_t>(sp.rt) * kTileRows + n_loc; kb = sp.k; }
-      else     { n = static_cast<int64_t>(sp.k) * kKStage + n_loc; kb = static_cast<int64_t>(sp.rt) * 2 + kb_loc; }
+      if (!dx) {
+        n = static_cast<int64_t>(sp.rt) * rows_per_tile + row_off + n_loc;
+        kb = sp.k;
+      } else {
+        n = static_cast<int64_t>(sp.k) * kKStage + n_loc;
+        kb = (static_cast<int64_t>(sp.rt) * rows_per_tile + row_off) / kBlock + kb_loc;
+      }
       if (n < p.N && kb < kb_row) {
         const int64_t b = n * kb_row + kb;
         q8 = __ldg(p.scale8 + b);
@@ -397,11 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t qv[3];
     float dv[3];
     StepPos pf;                    // position of the next prefetch
-    pf.init(g, p.nk, p.row_tiles);
+    pf.init(g, p.nk, walk);
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       scale_at(pf, 2 * u + g, qv[u], dv[u]);
-      pf.advance(2, p.nk, p.row_tiles);
+      pf.advance(2, p.nk, walk);
     }
     RingPos cr{g, 0}, ar{g, 0};    // rings of depth >= 2: step g sits in slot g of phase 0
     bool ok = true;
@@ -434,9 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.af[as]);
+        if (lane == 0) arrive_leader(&sm.af[as]);
         scale_at(pf, it + 6, qv[u], dv[u]);
-        pf.advance(2, p.nk, p.row_tiles);
+        pf.advance(2, p.nk, walk);
         cr.advance(2, p.sc);
         ar.advance(2, p.sa);
       }
@@ -445,9 +502,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync_all();   // the pair is done with each other's smem and TMEM
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_cols);
+    if constexpr (kPair) tmem_dealloc_pair(tmem_base, tmem_cols);
+    else tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 
@@ -456,9 +515,9 @@ CUtensorMapSwizzle lora_swizzle(int r_pad) {
                      : (r_pad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-size_t smem_bytes(int bt, int r_pad, int sx, int sa, int sc) {
-  return 1024 /* alignment slack */ + static_cast<size_t>(sx) * bt * 128u +
-         static_cast<size_t>(sa) * kATileBytes + lora_b_bytes(bt, r_pad) + lora_a_bytes(r_pad) +
+size_t smem_bytes(int bt_cta, int r_pad, int sx, int sa, int sc) {
+  return 1024 /* alignment slack */ + static_cast<size_t>(sx) * bt_cta * 128u +
+         static_cast<size_t>(sa) * kATileBytes + lora_b_bytes(bt_cta, r_pad) + lora_a_bytes(r_pad) +
          2 * kOutStageBytes + static_cast<size_t>(sc) * kCodeTileBytes +
          static_cast<size_t>(2 * (sx + sa + sc) + 7) * 8 + 16;
 }
@@ -466,12 +525,12 @@ size_t smem_bytes(int bt, int r_pad, int sx, int sa, int sc) {
 // Ring depths that fit the shared-memory budget, in order of preference: at
 // least four activation stages (TMA latency), codes several steps ahead, three
 // dequantised tiles ahead of the MMA.
-void pick_rings(int bt, int r_pad, int &sx, int &sa, int &sc) {
+void pick_rings(int bt_cta, int r_pad, int &sx, int &sa, int &sc) {
   const size_t budget = 227 * 1024;
   for (sx = 8; sx >= 4; --sx) {
     for (sc = 6; sc >= 4; sc -= 2) {
       sa = 3;
-      if (smem_bytes(bt, r_pad, sx, sa, sc) <= budget) return;
+      if (smem_bytes(bt_cta, r_pad, sx, sa, sc) <= budget) return;
     }
   }
   const int fallback[][3] = {{3, 3, 4}, {3, 2, 4}, {2, 2, 4}, {2, 2, 3}};
@@ -479,7 +538,7 @@ void pick_rings(int bt, int r_pad, int &sx, int &sa, int &sc) {
     sx = f[0];
     sa = f[1];
     sc = f[2];
-    if (smem_bytes(bt, r_pad, sx, sa, sc) <= budget) return;
+    if (smem_bytes(bt_cta, r_pad, sx, sa, sc) <= budget) return;
   }
 }
 
@@ -504,20 +563,25 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   else if (a.M <= 32) bt = 32;
   else if (a.M <= 64) bt = 64;
   else if (a.M <= 128) bt = 128;
+  // CTA pairs for the full 256-token tiles; single CTAs for short token counts.
+  const bool pair = false;   // the CTA-pair variant is kept but not dispatched: slower on B200
   p.bt = bt;
+  p.bt_cta = pair ? bt / 2 : bt;
   p.r_pad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
-  pick_rings(bt, p.r_pad, p.sx, p.sa, p.sc);
-  const int64_t rows = a.mode == 0 ? a.N : a.K;         // UMMA M extent
-  p.row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
+  pick_rings(p.bt_cta, p.r_pad, p.sx, p.sa, p.sc);
+  const int64_t rows = a.mode == 0 ? a.N : a.K;         // weight extent along UMMA M
+  const int rows_per_tile = pair ? 2 * kTileRows : kTileRows;
+  p.row_tiles = static_cast<int>((rows + rows_per_tile - 1) / rows_per_tile);
   p.tok_tiles = static_cast<int>((a.M + bt - 1) / bt);
   p.nk = static_cast<int>(a.mode == 0 ? a.K / kKStage : (a.N + kKStage - 1) / kKStage);
 
   CUtensorMap tm_act, tm_codes, tm_lw, tm_la, tm_out;
   const CUtensorMapSwizzle lsw = lora_swizzle(p.r_pad);
   const uint32_t box_t = bt < kEpiTokens ? bt : kEpiTokens;
+  const uint32_t bt_cta = static_cast<uint32_t>(p.bt_cta);
   bool ok = true;
   if (a.mode == 0) {
-    ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.K, a.M, a.K * 2, 64, bt,
+    ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.K, a.M, a.K * 2, 64, bt_cta,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= encode_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, a.K / 2, a.N, a.K / 2, 32,
                     kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -526,7 +590,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
     ok &= encode_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.N * 2, kTileRows,
                     box_t, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
-    ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.N, a.M, a.N * 2, 64, bt,
+    ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.N, a.M, a.N * 2, 64, bt_cta,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= encode_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, a.K / 2, a.N, a.K / 2, 64,
                     64, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -536,18 +600,38 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
                     box_t, CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   ok &= encode_2d(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lora_act, a.r, a.M, a.r * 2, p.r_pad,
-                  bt, lsw);
+                  bt_cta, lsw);
   if (!ok) return cudaErrorInvalidValue;
 
-  const size_t smem = smem_bytes(bt, p.r_pad, p.sx, p.sa, p.sc);
-  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  const size_t smem = smem_bytes(p.bt_cta, p.r_pad, p.sx, p.sa, p.sc);
   const int ntiles = p.row_tiles * p.tok_tiles;
   const int sms = device_sm_count();
-  const int grid = ntiles < sms ? ntiles : sms;
-  fused_nf4_gemm_kernel<<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, p);
-  return cudaGetLastError();
+  if (!pair) {
+    cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = ntiles < sms ? ntiles : sms;
+    fused_nf4_gemm_kernel<false><<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, p);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int pairs = ntiles < sms / 2 ? ntiles : sms / 2;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void *args[] = {&tm_act, &tm_codes, &tm_lw, &tm_la, &tm_out, &p};
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true>), args);
 }
 
 }  // namespace qlora
