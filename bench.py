@@ -182,6 +182,7 @@ def make_sets(q, torch, n_sets, N, K, M, r, outliers):
         d["dA"] = torch.empty((r, K), dtype=torch.float32, device="cuda")
         d["dB"] = torch.empty((N, r), dtype=torch.float32, device="cuda")
         d["ws"] = torch.empty(q.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+        d["gws"] = torch.empty(q.fused_workspace(M), dtype=torch.uint8, device="cuda")
         sets.append(d)
     torch.cuda.synchronize()
     return sets
@@ -196,19 +197,19 @@ def run_step(q, d, s, ev=None):
     q.lora_xa(d["X"], d["A"], s, d["sU"], d["ws"])
     if ev is not None:
         ev[0].record()
-    q.fused_fwd(d["q"], d["X"], d["B"], d["sU"], d["Y"])
+    q.fused_fwd(d["q"], d["X"], d["B"], d["sU"], d["Y"], ws=d["gws"])
     if ev is not None:
         ev[1].record()
     q.lora_dyb(d["dY"], d["B"], s, d["sT"], d["ws"])
     if ev is not None:
         ev[2].record()
-    q.fused_dx(d["q"], d["dY"], d["A"], d["sT"], d["dX"])
+    q.fused_dx(d["q"], d["dY"], d["A"], d["sT"], d["dX"], ws=d["gws"])
     if ev is not None:
         ev[3].record()
     q.lora_grads(d["X"], d["dY"], d["sU"], d["sT"], d["dA"], d["dB"], d["ws"])
 
 
-LAUNCHES_PER_STEP = 10   # lora_xa 2, fused_fwd 1, lora_dyb 2, fused_dx 1, lora_grads 4
+LAUNCHES_PER_STEP = 5   # lora_xa, fused_fwd, lora_dyb, fused_dx, lora_grads: one kernel each
 
 
 def profile_traffic(kernel_file_hash):
@@ -290,7 +291,8 @@ def bench_decode(q, torch, mats, steps, warmup):
             per_shape[key] = dict(X=X, Y=torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda"),
                                   sU=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
                                   ws=torch.empty(q.linear_workspace(M, lin.N, lin.K, r), dtype=torch.uint8,
-                                                 device="cuda"))
+                                                 device="cuda"),
+                                  gws=torch.empty(q.fused_workspace(M), dtype=torch.uint8, device="cuda"))
         A = (torch.randn((r, lin.K), generator=g, device="cuda") / r).to(torch.bfloat16)
         B = (torch.randn((lin.N, r), generator=g, device="cuda") * 0.01).to(torch.bfloat16)
         lora.append((A, B))
@@ -300,7 +302,7 @@ def bench_decode(q, torch, mats, steps, warmup):
         for (lin, m), (A, B) in zip(mats, lora):
             d = per_shape[(lin.N, lin.K)]
             q.lora_xa(d["X"], A, s, d["sU"], d["ws"])
-            q.fused_fwd(m, d["X"], B, d["sU"], d["Y"])
+            q.fused_fwd(m, d["X"], B, d["sU"], d["Y"], ws=d["gws"])
 
     for _ in range(warmup):
         one_pass()
@@ -313,7 +315,7 @@ def bench_decode(q, torch, mats, steps, warmup):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     return {"workload": "set_8b forward at 8 tokens: 224 matrices, r=16", "GB/s": moved / ms / 1e6,
-            "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": 3 * len(mats)}
+            "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": 2 * len(mats)}
 
 
 # ---------------------------------------------------------------------------

@@ -18,6 +18,7 @@ __all__ = [
     "nf4_sizes", "nf4_codebook", "nf4_quantize", "nf4_dequantize",
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
+    "fused_workspace",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -34,7 +35,7 @@ SYMBOLS = [
     "qlora_nf4_sizes", "qlora_nf4_codebook", "qlora_nf4_quantize", "qlora_nf4_dequantize",
     "qlora_linear_workspace", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
-    "qlora_linear_fwd_noalloc",
+    "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
 ]
 
 
@@ -91,9 +92,11 @@ def library():
     lib.qlora_lora_xa.restype = st
     lib.qlora_lora_dyb.argtypes = [_P, _I64, _I64, _P, ctypes.c_int32, ctypes.c_float, _P, _P, _SZ, _P]
     lib.qlora_lora_dyb.restype = st
-    lib.qlora_fused_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P]
+    lib.qlora_fused_workspace.argtypes = [_I64, ctypes.POINTER(_SZ)]
+    lib.qlora_fused_workspace.restype = st
+    lib.qlora_fused_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P, _P]
     lib.qlora_fused_fwd.restype = st
-    lib.qlora_fused_dx.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P]
+    lib.qlora_fused_dx.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P, _P]
     lib.qlora_fused_dx.restype = st
     lib.qlora_lora_grads.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P]
     lib.qlora_lora_grads.restype = st
@@ -251,19 +254,31 @@ def lora_dyb(dY, B, s: float, sT, ws, stream=None):
     return sT
 
 
-def fused_fwd(q: NF4Matrix, X, B, sU, Y, status=None, stream=None):
-    """Y = X W'^T + sU B^T (dequantisation fused into the tensor-core GEMM)."""
+def fused_workspace(M: int) -> int:
+    """Bytes of the optional stream-K workspace of fused_fwd / fused_dx."""
+    b = _SZ(0)
+    _check(library().qlora_fused_workspace(M, ctypes.byref(b)), "qlora_fused_workspace")
+    return b.value
+
+
+def _ws_args(ws):
+    return (None, 0) if ws is None else (_ptr(ws), ws.numel() * ws.element_size())
+
+
+def fused_fwd(q: NF4Matrix, X, B, sU, Y, status=None, stream=None, ws=None):
+    """Y = X W'^T + sU B^T (dequantisation fused into the tensor-core GEMM).
+    With `ws` (fused_workspace(M) bytes) the work is split stream-K over all SMs."""
     st = q.c_struct()
     _check(library().qlora_fused_fwd(ctypes.byref(st), _ptr(X), X.shape[0], _ptr(B), B.shape[1], _ptr(sU),
-                                     _ptr(Y), _ptr(status), _stream(stream)), "qlora_fused_fwd")
+                                     _ptr(Y), *_ws_args(ws), _ptr(status), _stream(stream)), "qlora_fused_fwd")
     return Y
 
 
-def fused_dx(q: NF4Matrix, dY, A, sT, dX, status=None, stream=None):
-    """dX = dY W' + sT A (dequantisation fused into the tensor-core GEMM)."""
+def fused_dx(q: NF4Matrix, dY, A, sT, dX, status=None, stream=None, ws=None):
+    """dX = dY W' + sT A (dequantisation fused into the tensor-core GEMM); `ws` as in fused_fwd."""
     st = q.c_struct()
     _check(library().qlora_fused_dx(ctypes.byref(st), _ptr(dY), dY.shape[0], _ptr(A), A.shape[0], _ptr(sT),
-                                    _ptr(dX), _ptr(status), _stream(stream)), "qlora_fused_dx")
+                                    _ptr(dX), *_ws_args(ws), _ptr(status), _stream(stream)), "qlora_fused_dx")
     return dX
 
 

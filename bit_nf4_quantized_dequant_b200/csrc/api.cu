@@ -59,8 +59,9 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, ui
 
 // Workspace layout of the linear calls (offsets in bytes, 256-byte aligned):
 //   [sU scratch: M*r bf16][sT: M*r bf16][fp32 partial sums of the skinny products]
+//   [stream-K workspace of the fused GEMMs]
 struct WsLayout {
-  size_t su, st, part, part_floats, total;
+  size_t su, st, part, part_floats, gemm, gemm_bytes, total;
 };
 
 static WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r) {
@@ -74,7 +75,9 @@ static WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r) {
   f = f > lora_cols_ws_floats(M, K, r) ? f : lora_cols_ws_floats(M, K, r);
   f = f > lora_cols_ws_floats(M, N, r) ? f : lora_cols_ws_floats(M, N, r);
   w.part_floats = f;
-  w.total = w.part + round_up(f * 4, 256);
+  w.gemm = w.part + round_up(f * 4, 256);
+  w.gemm_bytes = fused_gemm_ws_bytes(M);
+  w.total = w.gemm + round_up(w.gemm_bytes, 256);
   return w;
 }
 
@@ -178,13 +181,20 @@ qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const ui
                                       ws_bytes / 4, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_fused_workspace(int64_t M, size_t *bytes) {
+  if (!bytes || M < 1) return QLORA_ERR_INVALID_ARG;
+  *bytes = fused_gemm_ws_bytes(M);
+  return QLORA_OK;
+}
+
 static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act, int64_t M,
                             const uint16_t *lora_w, int32_t r, const uint16_t *lora_act, uint16_t *out,
-                            int32_t *dev_status, qlora_stream_t stream) {
+                            void *ws, size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
   qlora_status_t st = check_linear(W, act, M, lora_w, lora_w, r, 1.0f);
   if (st != QLORA_OK) return st;
   if (!lora_act || !out) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(lora_act) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
+  if (!aligned16(lora_act) || !aligned16(out) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
+  if (ws && ws_bytes < fused_gemm_ws_bytes(M)) return QLORA_ERR_WORKSPACE;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
   GemmArgs g{};
   g.mode = mode;
@@ -200,19 +210,20 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   g.lora_act = lora_act;
   g.out = out;
   g.dev_status = dev_status;
+  g.ws = ws;
   return cuda_status(launch_fused_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qlora_status_t qlora_fused_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *B,
-                               int32_t r, const uint16_t *sU, uint16_t *Y, int32_t *dev_status,
-                               qlora_stream_t stream) {
-  return fused(0, W, X, M, B, r, sU, Y, dev_status, stream);
+                               int32_t r, const uint16_t *sU, uint16_t *Y, void *ws, size_t ws_bytes,
+                               int32_t *dev_status, qlora_stream_t stream) {
+  return fused(0, W, X, M, B, r, sU, Y, ws, ws_bytes, dev_status, stream);
 }
 
 qlora_status_t qlora_fused_dx(const qlora_nf4_t *W, const uint16_t *dY, int64_t M, const uint16_t *A,
-                              int32_t r, const uint16_t *sT, uint16_t *dX, int32_t *dev_status,
-                              qlora_stream_t stream) {
-  return fused(1, W, dY, M, A, r, sT, dX, dev_status, stream);
+                              int32_t r, const uint16_t *sT, uint16_t *dX, void *ws, size_t ws_bytes,
+                              int32_t *dev_status, qlora_stream_t stream) {
+  return fused(1, W, dY, M, A, r, sT, dX, ws, ws_bytes, dev_status, stream);
 }
 
 qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
@@ -244,7 +255,7 @@ qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(wsb + L.su);
   st = qlora_lora_xa(X, M, K, A, r, s, sU, wsb + L.part, L.part_floats * 4, stream);
   if (st != QLORA_OK) return st;
-  return qlora_fused_fwd(W, X, M, B, r, sU, Y, dev_status, stream);
+  return qlora_fused_fwd(W, X, M, B, r, sU, Y, wsb + L.gemm, L.gemm_bytes, dev_status, stream);
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
@@ -275,7 +286,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   st = qlora_lora_dyb(dY, M, N, B, r, s, sT, part, part_bytes, stream);
   if (st != QLORA_OK) return st;
   if (dX) {
-    st = qlora_fused_dx(W, dY, M, A, r, sT, dX, dev_status, stream);
+    st = qlora_fused_dx(W, dY, M, A, r, sT, dX, wsb + L.gemm, L.gemm_bytes, dev_status, stream);
     if (st != QLORA_OK) return st;
   }
   return qlora_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, part, part_bytes, stream);

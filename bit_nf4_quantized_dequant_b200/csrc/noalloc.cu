@@ -73,5 +73,5 @@ extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const u
   uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(base);
   st = qlora_lora_xa(X, M, W->cols, A, r, s, sU, base + su_bytes, part_bytes, stream);
   if (st != QLORA_OK) return st;
-  return qlora_fused_fwd(W, X, M, B, r, sU, Y, dev_status, stream);
+  return qlora_fused_fwd(W, X, M, B, r, sU, Y, nullptr, 0, dev_status, stream);   // whole-tile schedule
 }

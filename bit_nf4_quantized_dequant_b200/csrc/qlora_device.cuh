@@ -176,9 +176,37 @@ __device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_
                : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` (multiple of 16, both addresses
+// 16-byte aligned) that completes transaction bytes on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(sdst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Orders this thread's completed async-proxy (bulk copy) writes to global
+// memory before its later generic-proxy accesses, such as a release store.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Barrier over a subset of the CTA's warps (id 1..15, count a multiple of 32).
+// bar.sync is an aligned barrier: every lane of a warp must arrive together,
+// so the warp is reconverged first (lanes may come from a single-lane branch).
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Flag publication between CTAs of one grid (global memory, GPU scope).
+__device__ __forceinline__ void st_release_gpu_u64(uint64_t *p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tcgen05).
@@ -192,8 +220,10 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-// All threads of all CTAs of the cluster (release / acquire).
+// All threads of all CTAs of the cluster (release / acquire). The barrier is
+// aligned, so each warp is reconverged before it arrives.
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");

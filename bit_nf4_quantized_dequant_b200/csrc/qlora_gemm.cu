@@ -26,11 +26,17 @@
 //
 // Two variants share this source. Single CTA: UMMA M = 128, one CTA per tile.
 // CTA pair (cta_group::2, a cluster of two): UMMA M = 256 across the pair; each
-// CTA dequantises its own 128 weight rows and loads half of the token tile, and
-// the pair's tensor cores read both halves, so every SM moves about a third
-// less data through shared memory per flop. The even CTA issues the MMAs; the
-// odd CTA's producers and dequantisers signal the even CTA's barriers, and the
-// even CTA's MMA completions are multicast to both.
+// CTA dequantises its own 128 weight rows and loads half of the token tile.
+// The even CTA issues the MMAs; the odd CTA's producers and dequantisers signal
+// the even CTA's barriers, and the even CTA's MMA completions are multicast to
+// both. The pair halves each SM's activation traffic, but that traffic is not
+// what limits this kernel, and the cluster-scope arrivals cost more than they
+// save, so the launcher dispatches the single-CTA variant.
+//
+// Scheduling: persistent CTAs take whole tiles (tile = blockIdx + i * gridDim).
+// With a workspace and token tiles of at most 64, stream-K instead: the
+// (tile, k-step) units are split evenly over all SMs, and tiles cut between
+// CTAs are finished through fp32 partials in the workspace (see GemmParams).
 //
 // Warp roles (512 threads): 0 codes producer, 1 MMA issuer and TMEM owner,
 // 2 activation producer, 3 LoRA-slice producer, 4-7 epilogue (TMEM lane
@@ -38,6 +44,8 @@
 // 8-11 and 12-15 the two dequantiser groups. Persistent CTAs walk the tile
 // list; the TMEM accumulator is double-buffered so the epilogue of one tile
 // overlaps the main loop of the next.
+#include <atomic>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
@@ -64,6 +72,17 @@ struct GemmParams {
   int row_tiles;   // tiles along the weight dimension (128 rows, or 256 for a pair)
   int tok_tiles;
   int nk;          // main-loop K steps per tile
+  // Stream-K (single CTA only): CTA b of G takes units [b*U/G, (b+1)*U/G) of
+  // the U = tiles * nk (tile, k-step) units. A tile split between CTAs is
+  // finished by the CTA that holds its k = 0 unit (the lowest one); every
+  // other CTA working on the tile has it as its first segment and publishes
+  // that partial (fp32, part + j * 128 * bt, column-major [bt][128]) by
+  // setting flags[j] = epoch, a value unique to the launch. The finishing CTA
+  // adds the partials in CTA order and clears the flags for the next launch.
+  int streamk;
+  uint64_t epoch;
+  float *part;
+  uint64_t *flags;
 };
 
 __host__ __device__ inline uint32_t lora_a_bytes(int r_pad) { return kTileRows * r_pad * 2; }
@@ -78,7 +97,7 @@ __device__ __forceinline__ uint32_t lora_layout(int r_pad) {
 struct Smem {
   uint8_t *x, *a, *lb, *la, *out, *c;
   uint32_t x_bytes;
-  uint64_t *xf, *xe, *af, *ae, *cf, *ce, *lf, *le, *accf, *acce, *drain;
+  uint64_t *xf, *xe, *af, *ae, *cf, *ce, *lf, *le, *accf, *acce, *drain, *peer_full;
   uint32_t *tmem_holder;
   int *abort_flag;
 };
@@ -100,7 +119,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmParams &p) {
   s.lf = s.ce + p.sc; s.le = s.lf + 1;
   s.accf = s.le + 1;  s.acce = s.accf + 2;
   s.drain = s.acce + 2;
-  s.tmem_holder = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.peer_full = s.drain + 1;
+  s.tmem_holder = reinterpret_cast<uint32_t *>(s.peer_full + 1);
   s.abort_flag = reinterpret_cast<int *>(s.tmem_holder + 1);
   return s;
 }
@@ -118,31 +138,33 @@ struct RingPos {
   }
 };
 
-// Which tiles a CTA (or CTA pair) walks: tile = first + lt * stride.
-struct TileWalk {
-  int first, stride, row_tiles;
+// The (tile, k-step) units a CTA (or CTA pair) processes, in order: starting at
+// (first_tile, first_k), k runs to nk and then continues at k = 0 of tile +
+// stride, for `total` units. Data-parallel: first_k = 0, stride = CTA count,
+// whole tiles. Stream-K: stride = 1 over a contiguous range of units.
+struct Walk {
+  int first_tile, first_k, stride, total, row_tiles;
 };
 
-// (local tile, k-step) of a position in this CTA's step sequence, advanced
-// without division; rt / tt are the tile's indices along weights / tokens.
+// A position in a Walk, advanced without division; rt / tt are the tile's
+// indices along weights / tokens.
 struct StepPos {
-  int lt, k, rt, tt;
-  __device__ __forceinline__ void set_tile(const TileWalk &w) {
-    const int tile = w.first + lt * w.stride;
+  int tile, k, rt, tt;
+  __device__ __forceinline__ void set_tile(const Walk &w) {
     rt = tile % w.row_tiles;
     tt = tile / w.row_tiles;
   }
-  __device__ __forceinline__ void init(int it, int nk, const TileWalk &w) {
-    lt = it / nk;
-    k = it - lt * nk;
+  __device__ __forceinline__ void init(const Walk &w) {
+    tile = w.first_tile;
+    k = w.first_k;
     set_tile(w);
   }
-  __device__ __forceinline__ void advance(int by, int nk, const TileWalk &w) {
+  __device__ __forceinline__ void advance(int by, int nk, const Walk &w) {
     k += by;
     if (k >= nk) {
       while (k >= nk) {
         k -= nk;
-        ++lt;
+        tile += w.stride;
       }
       set_tile(w);
     }
@@ -177,11 +199,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTA pair: rank 0 (even CTA) issues the MMAs; rank 1 is its peer.
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
-  const TileWalk walk{kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x),
-                      kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x), p.row_tiles};
   const int ntiles = p.row_tiles * p.tok_tiles;
-  const int nlt = ntiles > walk.first ? (ntiles - walk.first + walk.stride - 1) / walk.stride : 0;
-  const int total_steps = nlt * p.nk;
+  Walk walk;
+  walk.row_tiles = p.row_tiles;
+  const int64_t units = static_cast<int64_t>(ntiles) * p.nk;
+  // first unit of CTA j under the stream-K split
+  auto unit_begin = [&](int64_t j) -> int64_t { return units * j / gridDim.x; };
+  if (!kPair && p.streamk) {
+    const int64_t u0 = unit_begin(blockIdx.x), u1 = unit_begin(blockIdx.x + 1);
+    walk.first_tile = static_cast<int>(u0 / p.nk);
+    walk.first_k = static_cast<int>(u0 % p.nk);
+    walk.stride = 1;
+    walk.total = static_cast<int>(u1 - u0);
+  } else {
+    const int first = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int stride = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const int nlt = ntiles > first ? (ntiles - first + stride - 1) / stride : 0;
+    walk.first_tile = first;
+    walk.first_k = 0;
+    walk.stride = stride;
+    walk.total = nlt * p.nk;
+  }
+  const int total_steps = walk.total;
   const int rows_per_tile = kPair ? 2 * kTileRows : kTileRows;
   const int row_off = static_cast<int>(rank) * kTileRows;     // this CTA's weight rows inside the tile
   const int tok_off = static_cast<int>(rank) * p.bt_cta;      // this CTA's tokens inside the tile
@@ -198,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sm.le, 1);
     for (int i = 0; i < 2; ++i) { mbar_init(&sm.accf[i], 1); mbar_init(&sm.acce[i], per_step); }
     mbar_init(sm.drain, 1);
+    mbar_init(sm.peer_full, 1);
     *sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -244,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       RingPos c{0, 0};
       StepPos sp;
-      sp.init(0, p.nk, walk);
+      sp.init(walk);
       for (int it = 0; it < total_steps; ++it, c.advance(1, p.sc), sp.advance(1, p.nk, walk)) {
         const int s = c.slot;
         const uint32_t ph = c.phase;
@@ -266,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       RingPos x{0, 0};
       StepPos sp;
-      sp.init(0, p.nk, walk);
+      sp.init(walk);
       for (int it = 0; it < total_steps; ++it, x.advance(1, p.sx), sp.advance(1, p.nk, walk)) {
         const int s = x.slot;
         const uint32_t ph = x.phase;
@@ -285,22 +325,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued = false;
       uint32_t last_ph = 0;
       const uint32_t bytes_cta = lora_a_bytes(p.r_pad) + static_cast<uint32_t>(p.bt_cta) * p.r_pad * 2u;
-      for (int lt = 0; lt < nlt; ++lt) {
-        const int tile = walk.first + lt * walk.stride;
-        const int rt = tile % p.row_tiles, tt = tile / p.row_tiles;
-        const int r0 = rt * rows_per_tile + row_off;
-        const uint32_t ph = static_cast<uint32_t>(lt) & 1u;
-        if (!mbar_wait(sm.le, ph ^ 1u, abort_flag, p.status)) break;
-        if (leader) mbar_arrive_expect_tx(sm.lf, kPair ? 2 * bytes_cta : bytes_cta);
-        load_for_leader(sm.lb, &tm_lora_act, sm.lf, 0, tt * p.bt + tok_off);
-        if (!dx) {
-          load_for_leader(sm.la, &tm_lora_w, sm.lf, 0, r0);
-        } else {
-          load_for_leader(sm.la, &tm_lora_w, sm.lf, r0, 0);
-          load_for_leader(sm.la + p.r_pad * 128, &tm_lora_w, sm.lf, r0 + 64, 0);
+      StepPos seg;
+      seg.init(walk);
+      int n_lora = 0;
+      for (int done = 0; done < total_steps;) {
+        const int len = p.nk - seg.k < total_steps - done ? p.nk - seg.k : total_steps - done;
+        if (seg.k + len == p.nk) {   // this segment ends its tile: it carries the LoRA K-steps
+          const int r0 = seg.rt * rows_per_tile + row_off;
+          const uint32_t ph = static_cast<uint32_t>(n_lora) & 1u;
+          if (!mbar_wait(sm.le, ph ^ 1u, abort_flag, p.status)) break;
+          if (leader) mbar_arrive_expect_tx(sm.lf, kPair ? 2 * bytes_cta : bytes_cta);
+          load_for_leader(sm.lb, &tm_lora_act, sm.lf, 0, seg.tt * p.bt + tok_off);
+          if (!dx) {
+            load_for_leader(sm.la, &tm_lora_w, sm.lf, 0, r0);
+          } else {
+            load_for_leader(sm.la, &tm_lora_w, sm.lf, r0, 0);
+            load_for_leader(sm.la + p.r_pad * 128, &tm_lora_w, sm.lf, r0 + 64, 0);
+          }
+          issued = true;
+          last_ph = ph;
+          ++n_lora;
         }
-        issued = true;
-        last_ph = ph;
+        done += len;
+        seg.advance(len, p.nk, walk);
       }
       if (*abort_flag && issued && leader) drain_ring(sm.lf, 1, 1u, last_ph);
     }
@@ -327,15 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_step = dx ? 2048u / 16u : 32u / 16u;
       bool ok = true, issued_any = false;
       RingPos xr{0, 0}, ar{0, 0};
-      for (int lt = 0; lt < nlt && ok; ++lt) {
-        const int buf = lt & 1;
-        if (!mbar_wait(&sm.acce[buf], (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
+      StepPos seg;
+      seg.init(walk);
+      int n_lora = 0;
+      for (int done = 0, si = 0; done < total_steps && ok; ++si) {
+        const int kb = seg.k;
+        const int len = p.nk - kb < total_steps - done ? p.nk - kb : total_steps - done;
+        const int buf = si & 1;
+        if (!mbar_wait(&sm.acce[buf], (static_cast<uint32_t>(si >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * p.bt);
-        for (int k = 0; k < p.nk; ++k, xr.advance(1, p.sx), ar.advance(1, p.sa)) {
+        for (int k = 0; k < len; ++k, xr.advance(1, p.sx), ar.advance(1, p.sa)) {
           const int xs = xr.slot, as = ar.slot;
           if (!mbar_wait(&sm.xf[xs], xr.phase, abort_flag, p.status) ||
               !mbar_wait(&sm.af[as], ar.phase, abort_flag, p.status)) {
@@ -355,17 +407,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit(&sm.ae[as]);
         }
         if (!ok) break;
-        // LoRA K-steps: [.. | B] x [.. | sU] (FWD) or [.. ; A] x [.. | sT] (DX)
-        if (!mbar_wait(sm.lf, static_cast<uint32_t>(lt) & 1u, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        for (int j = 0; j < p.r_pad / 16; ++j) {
-          const uint64_t ad = dx ? smem_desc(la_addr + 2048u * j, 128u * p.r_pad, 1024u, kLayoutSW128)
-                                 : smem_desc(la_addr + 32u * j, 16u, lsbo, lsw);
-          const uint64_t bd = smem_desc(lb_addr + 32u * j, 16u, lsbo, lsw);
-          mma(d_tmem, ad, bd, 1u);
+        if (kb + len == p.nk) {
+          // LoRA K-steps: [.. | B] x [.. | sU] (FWD) or [.. ; A] x [.. | sT] (DX)
+          if (!mbar_wait(sm.lf, static_cast<uint32_t>(n_lora) & 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          for (int j = 0; j < p.r_pad / 16; ++j) {
+            const uint64_t ad = dx ? smem_desc(la_addr + 2048u * j, 128u * p.r_pad, 1024u, kLayoutSW128)
+                                   : smem_desc(la_addr + 32u * j, 16u, lsbo, lsw);
+            const uint64_t bd = smem_desc(lb_addr + 32u * j, 16u, lsbo, lsw);
+            mma(d_tmem, ad, bd, 1u);
+          }
+          commit(sm.le);
+          ++n_lora;
         }
-        commit(sm.le);
         commit(&sm.accf[buf]);
+        done += len;
+        seg.advance(len, p.nk, walk);
       }
       if (!ok && issued_any) {
         // drain: wait until every MMA issued so far has finished reading/writing
@@ -382,38 +439,143 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int box_t = p.bt < kEpiTokens ? p.bt : kEpiTokens;
     const int nchunks = p.bt / box_t;
     uint32_t chunk_count = 0;
-    for (int lt = 0; lt < nlt; ++lt) {
-      const int tile = walk.first + lt * walk.stride;
-      const int rt = tile % p.row_tiles, tt = tile / p.row_tiles;
-      const int buf = lt & 1;
-      if (!mbar_wait(&sm.accf[buf], static_cast<uint32_t>(lt >> 1) & 1u, abort_flag, p.status)) break;
+    StepPos seg;
+    seg.init(walk);
+    const int64_t part_elems = static_cast<int64_t>(kTileRows) * p.bt;
+    for (int done = 0, si = 0; done < total_steps; ++si) {
+      const int kb = seg.k;
+      const int len = p.nk - kb < total_steps - done ? p.nk - kb : total_steps - done;
+      const int rt = seg.rt, tt = seg.tt;
+      const bool head = kb > 0;                  // the end of a tile whose start another CTA computes
+      const bool tail = kb + len < p.nk;         // the start of a tile that the next CTA completes
+      const int buf = si & 1;
+      if (!mbar_wait(&sm.accf[buf], static_cast<uint32_t>(si >> 1) & 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.bt);
-      for (int c = 0; c < nchunks; ++c, ++chunk_count) {
-        uint32_t v[32];
-        tmem_ld32(taddr + static_cast<uint32_t>(c * box_t), v);
-        tmem_ld_wait();
-        if (c == nchunks - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) arrive_leader(&sm.acce[buf]);
-        }
-        uint16_t *stage = reinterpret_cast<uint16_t *>(sm.out + (chunk_count & 1u) * kOutStageBytes);
-        if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
-        named_barrier(1, 128);
+      if (head) {
+        // Publish this partial accumulator for the CTA that finishes the tile:
+        // fp32, column-major [bt][128], staged chunk by chunk through the
+        // (otherwise idle: a head is a CTA's first segment) output buffer and
+        // written with bulk copies.
+        float *dst = p.part + static_cast<int64_t>(blockIdx.x) * part_elems;
+        float *stagef = reinterpret_cast<float *>(sm.out);
+        const uint32_t chunk_bytes = static_cast<uint32_t>(box_t) * kTileRows * 4u;
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + static_cast<uint32_t>(c * box_t), v);
+          tmem_ld_wait();
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_leader(&sm.acce[buf]);
+          }
+          if (et == 0) bulk_wait_group_read<0>();   // the previous chunk's copy has left the buffer
+          named_barrier(1, 128);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < box_t)
-            stage[j * kTileRows + et] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+          for (int j = 0; j < 32; ++j)
+            if (j < box_t) stagef[j * kTileRows + et] = __uint_as_float(v[j]);
+          fence_proxy_async_smem();
+          named_barrier(1, 128);
+          if (et == 0) {
+            bulk_store(dst + static_cast<int64_t>(c * box_t) * kTileRows, stagef, chunk_bytes);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
-        fence_proxy_async_smem();
-        named_barrier(1, 128);
         if (et == 0) {
-          tma_store_2d(&tm_out, stage, rt * rows_per_tile + row_off, tt * p.bt + c * box_t);
-          bulk_commit_group();
+          bulk_wait_group<0>();        // the partial is in global memory
+          fence_proxy_async_global();
+          __threadfence();
+          st_release_gpu_u64(p.flags + blockIdx.x, p.epoch);
+        }
+        __syncwarp();
+      } else {
+        // tail: CTAs blockIdx.x + 1 .. blockIdx.x + n_peers hold the rest of this tile
+        int n_peers = 0, n_smem = 0;
+        const float *peer = p.part + static_cast<int64_t>(blockIdx.x + 1) * part_elems;
+        const float *peer_s = reinterpret_cast<const float *>(sm.x);
+        if (tail) {
+          const int64_t tile_end = static_cast<int64_t>(seg.tile + 1) * p.nk;
+          while (static_cast<int64_t>(blockIdx.x) + n_peers + 1 < gridDim.x &&
+                 unit_begin(blockIdx.x + n_peers + 1) < tile_end)
+            ++n_peers;
+          // This is the CTA's last segment: its rings are idle, so the peers'
+          // partials are brought into them with bulk copies (as many as fit;
+          // any others are read from global memory).
+          const uint32_t part_bytes = static_cast<uint32_t>(part_elems) * 4u;
+          const int cap = static_cast<int>(static_cast<uint32_t>(sm.out - sm.x) / part_bytes);
+          n_smem = n_peers < cap ? n_peers : cap;
+          if (et == 0) {
+            const uint64_t t0 = global_timer_ns();
+            for (int j = 1; j <= n_peers; ++j) {
+              uint64_t *flag = p.flags + blockIdx.x + j;
+              while (ld_acquire_gpu_u64(flag) != p.epoch) {
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                  *abort_flag = 1;
+                  set_status(p.status, 6 /* QLORA_ERR_TIMEOUT */);
+                  break;
+                }
+                __nanosleep(256);
+              }
+              *flag = 0;   // consumed: the next launch (same epoch under graph replay) waits again
+            }
+            __threadfence();
+            fence_proxy_async_global();
+            if (n_smem > 0) {
+              mbar_arrive_expect_tx(sm.peer_full, part_bytes * static_cast<uint32_t>(n_smem));
+              for (int j = 0; j < n_smem; ++j)
+                bulk_load(sm.x + static_cast<size_t>(j) * part_bytes, peer + static_cast<int64_t>(j) * part_elems,
+                          part_bytes, sm.peer_full);
+            }
+          }
+          __syncwarp();
+          if (n_smem > 0) mbar_wait(sm.peer_full, 0, abort_flag, p.status);
+          named_barrier(1, 128);
+          __threadfence();
+        }
+        for (int c = 0; c < nchunks; ++c, ++chunk_count) {
+          uint32_t v[32];
+          tmem_ld32(taddr + static_cast<uint32_t>(c * box_t), v);
+          tmem_ld_wait();
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_leader(&sm.acce[buf]);
+          }
+          if (n_peers > 0) {
+            const int64_t off = static_cast<int64_t>(c * box_t) * kTileRows + et;
+            for (int pj = 0; pj < n_smem; ++pj) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < box_t)
+                  v[j] = __float_as_uint(__uint_as_float(v[j]) + peer_s[pj * part_elems + off + j * kTileRows]);
+            }
+            for (int pj = n_smem; pj < n_peers; ++pj) {
+              float w[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) w[j] = j < box_t ? __ldcg(peer + pj * part_elems + off + j * kTileRows) : 0.f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + w[j]);
+            }
+          }
+          uint16_t *stage = reinterpret_cast<uint16_t *>(sm.out + (chunk_count & 1u) * kOutStageBytes);
+          if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
+          named_barrier(1, 128);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < box_t) stage[j * kTileRows + et] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+          fence_proxy_async_smem();
+          named_barrier(1, 128);
+          if (et == 0) {
+            tma_store_2d(&tm_out, stage, rt * rows_per_tile + row_off, tt * p.bt + c * box_t);
+            bulk_commit_group();
+          }
+          __syncwarp();   // reconverge before the next warp-wide TMEM load
         }
       }
+      done += len;
+      seg.advance(len, p.nk, walk);
     }
     if (et == 0) bulk_wait_group<0>();
   } else {
@@ -454,7 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t qv[3];
     float dv[3];
     StepPos pf;                    // position of the next prefetch
-    pf.init(g, p.nk, walk);
+    pf.init(walk);
+    pf.advance(g, p.nk, walk);
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
       scale_at(pf, 2 * u + g, qv[u], dv[u]);
@@ -500,6 +663,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // Every role above ran on one elected lane (or left its loop on its own); the
+  // warp is reconverged before the CTA barrier (an aligned barrier) and before
+  // the warp-wide TMEM deallocation.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) cluster_sync_all();   // the pair is done with each other's smem and TMEM
@@ -519,7 +686,7 @@ size_t smem_bytes(int bt_cta, int r_pad, int sx, int sa, int sc) {
   return 1024 /* alignment slack */ + static_cast<size_t>(sx) * bt_cta * 128u +
          static_cast<size_t>(sa) * kATileBytes + lora_b_bytes(bt_cta, r_pad) + lora_a_bytes(r_pad) +
          2 * kOutStageBytes + static_cast<size_t>(sc) * kCodeTileBytes +
-         static_cast<size_t>(2 * (sx + sa + sc) + 7) * 8 + 16;
+         static_cast<size_t>(2 * (sx + sa + sc) + 8) * 8 + 16;
 }
 
 // Ring depths that fit the shared-memory budget, in order of preference: at
@@ -549,6 +716,22 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, ui
                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                CUtensorMapSwizzle swizzle);
 
+namespace {
+int token_tile(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+}  // namespace
+
+size_t fused_gemm_ws_bytes(int64_t M) {
+  const size_t sms = static_cast<size_t>(device_sm_count());
+  const size_t flags = (sms * 8 + 255) / 256 * 256;
+  return flags + sms * kTileRows * static_cast<size_t>(token_tile(M)) * 4;
+}
+
 cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   GemmParams p{};
   p.scale8 = a.scale8;
@@ -558,13 +741,10 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   p.K = a.K;
   p.M = a.M;
   p.mode = a.mode;
-  int bt = 256;
-  if (a.M <= 16) bt = 16;
-  else if (a.M <= 32) bt = 32;
-  else if (a.M <= 64) bt = 64;
-  else if (a.M <= 128) bt = 128;
-  // CTA pairs for the full 256-token tiles; single CTAs for short token counts.
-  const bool pair = false;   // the CTA-pair variant is kept but not dispatched: slower on B200
+  const int bt = token_tile(a.M);
+  // The CTA-pair variant is compiled but not dispatched: on B200 its remote
+  // barrier arrivals cost more than the shared-memory traffic it saves.
+  const bool pair = false;
   p.bt = bt;
   p.bt_cta = pair ? bt / 2 : bt;
   p.r_pad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
@@ -610,7 +790,21 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int grid = ntiles < sms ? ntiles : sms;
+    int grid = ntiles < sms ? ntiles : sms;
+    if (a.ws && bt <= 64) {
+      // Stream-K over all SMs for short token tiles: a few weight-row tiles
+      // would otherwise occupy a few SMs, and the fp32 partials that cross
+      // CTAs are small. With 128- and 256-token tiles the partials (64 and
+      // 128 KiB per split tile) cost more than the balance gains on B200.
+      const int64_t units = static_cast<int64_t>(ntiles) * p.nk;
+      grid = units < sms ? static_cast<int>(units) : sms;
+      static std::atomic<uint64_t> launch_counter{0x51C0FFEE00000000ull};
+      p.streamk = 1;
+      p.epoch = ++launch_counter;
+      const size_t flags = (static_cast<size_t>(sms) * 8 + 255) / 256 * 256;
+      p.flags = static_cast<uint64_t *>(a.ws);
+      p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + flags);
+    }
     fused_nf4_gemm_kernel<false><<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, p);
     return cudaGetLastError();
   }

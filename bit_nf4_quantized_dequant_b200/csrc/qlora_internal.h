@@ -30,8 +30,11 @@ struct GemmArgs {
   const uint16_t *lora_act; // sU or sT [M, r]
   uint16_t *out;            // Y [M, N] or dX [M, K]
   int32_t *dev_status;
+  void *ws;                 // optional stream-K workspace (fused_gemm_ws_bytes(M) bytes), or null
 };
 cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t s);
+// Workspace of a stream-K launch with M tokens on the current device.
+size_t fused_gemm_ws_bytes(int64_t M);
 
 // Skinny LoRA products (fp32 accumulation).
 // out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if

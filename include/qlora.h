@@ -149,8 +149,10 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
  * qlora_fused_dx and qlora_lora_grads (and qlora_lora_xa when sU is not
  * given). They are exposed so that a caller can schedule or time the steps
  * separately; arguments, layouts and errors are as in the composite calls.
- * `ws` is a workspace of at least qlora_linear_workspace() bytes for the same
- * (M, N, K, r); it only holds partial sums between the two kernels of a step.
+ * For the skinny products `ws` is a workspace of at least qlora_linear_workspace()
+ * bytes for the same (M, N, K, r) (they need none at present; the argument is
+ * kept so that a split of their reduction can use it). qlora_fused_workspace()
+ * sizes the optional workspace of the two fused GEMMs.
  */
 
 /* sU = bf16_rn(s X A^T), [M, r]. The adapter's down projection, the first
@@ -159,13 +161,27 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
 qlora_status_t qlora_lora_xa(const uint16_t *X, int64_t M, int64_t K, const uint16_t *A, int32_t r,
                              float s, uint16_t *sU, void *ws, size_t ws_bytes, qlora_stream_t stream);
 
+/* Bytes of the optional workspace of qlora_fused_fwd / qlora_fused_dx for M
+ * tokens on the current device (it scales with the device's SM count).
+ * Errors: INVALID_ARG (M < 1 or bytes NULL), CUDA. */
+qlora_status_t qlora_fused_workspace(int64_t M, size_t *bytes);
+
 /* Y = X W'^T + sU B^T with W' dequantised tile by tile in shared memory and
  * fed to the tensor cores; the LoRA term is one extra K-step of the same
  * accumulation ("QLoRA and Fine-Tuning on One Consumer GPU", "The idea in one
- * line"). Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+ * line").
+ * ws / ws_bytes: NULL / 0, or device memory of at least qlora_fused_workspace(M)
+ *   bytes, 16-byte aligned. With NULL every CTA takes whole output tiles. With a
+ *   workspace and M <= 64 (where whole tiles would leave most SMs idle) the
+ *   (tile, K-step) work is split evenly over all SMs and tiles cut between CTAs
+ *   are summed through fp32 partials kept there (results equal up to fp32
+ *   rounding order); larger M keeps whole tiles. The workspace needs no
+ *   initialisation and keeps no state the caller sees; one launch at a time may
+ *   use a given workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
 qlora_status_t qlora_fused_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *B,
-                               int32_t r, const uint16_t *sU, uint16_t *Y, int32_t *dev_status,
-                               qlora_stream_t stream);
+                               int32_t r, const uint16_t *sU, uint16_t *Y, void *ws, size_t ws_bytes,
+                               int32_t *dev_status, qlora_stream_t stream);
 
 /* sT = bf16_rn(s dY B), [M, r]: the gradient reaching the adapter's
  * bottleneck. N % 16 == 0. Errors: as qlora_lora_xa. */
@@ -173,10 +189,11 @@ qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const ui
                               float s, uint16_t *sT, void *ws, size_t ws_bytes, qlora_stream_t stream);
 
 /* dX = dY W' + sT A, [M, K] bf16, W' dequantised in shared memory as in
- * qlora_fused_fwd (here consumed untransposed). Errors: as qlora_fused_fwd. */
+ * qlora_fused_fwd (here consumed untransposed); ws as in qlora_fused_fwd.
+ * Errors: as qlora_fused_fwd. */
 qlora_status_t qlora_fused_dx(const qlora_nf4_t *W, const uint16_t *dY, int64_t M, const uint16_t *A,
-                              int32_t r, const uint16_t *sT, uint16_t *dX, int32_t *dev_status,
-                              qlora_stream_t stream);
+                              int32_t r, const uint16_t *sT, uint16_t *dX, void *ws, size_t ws_bytes,
+                              int32_t *dev_status, qlora_stream_t stream);
 
 /* dA = sT^T X ([r, K] fp32) and dB = dY^T sU ([N, r] fp32), both overwritten:
  * the adapter gradients ("QLoRA, in depth", "The mechanism in brief").

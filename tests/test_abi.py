@@ -90,6 +90,23 @@ def test_argument_errors_are_returned_before_any_launch(lib):
     assert so.qlora_linear_workspace(8, 32, 64, 16, None) == 1
     ws = SZ()
     assert so.qlora_linear_workspace(8, 32, 100, 16, ctypes.byref(ws)) == 2
+    # fused GEMMs: the optional stream-K workspace is checked before any launch
+    assert so.qlora_fused_workspace(0, ctypes.byref(ws)) == 1
+    assert so.qlora_fused_workspace(8, None) == 1
+    assert so.qlora_fused_workspace(8, ctypes.byref(ws)) == 0 and ws.value > 0
+    need = ws.value
+    sU, WS = P(0x90000), P(0xC0000)
+    assert so.qlora_fused_fwd(ctypes.byref(q), X, 8, B, 16, sU, Y, WS, need - 1, None, None) == 4
+    assert so.qlora_fused_dx(ctypes.byref(q), X, 8, A, 16, sU, Y, WS, need - 1, None, None) == 4
+    assert so.qlora_fused_fwd(ctypes.byref(q), X, 8, B, 16, sU, Y, P(0xC0008), need, None, None) == 3
+
+
+def test_fused_workspace_scales_with_token_tile(lib):
+    """Stream-K partials hold one [128 x token-tile] fp32 tile per SM: the size
+    grows with the token tile (16 .. 256 tokens) and then stays flat."""
+    sizes = [lib.fused_workspace(m) for m in (1, 16, 17, 128, 256, 4096)]
+    assert sizes[0] == sizes[1] < sizes[2] < sizes[3] < sizes[4] == sizes[5]
+    assert lib.linear_workspace(2048, 4096, 4096, 16) > lib.fused_workspace(2048)
 
 
 def test_workspace_grows_with_tokens(lib):

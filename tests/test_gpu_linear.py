@@ -117,3 +117,81 @@ def test_no_timeout_status(lib):
     lib.linear_bwd(d["q"], d["X"], d["A"], d["B"], 2.0, d["dY"], status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+
+
+# Shapes for the two schedules of the fused GEMMs: tiles split over many CTAs
+# (fewer tiles than SMs), a ragged second wave (more tiles than SMs), decode.
+# With a workspace, token tiles of at most 64 (M <= 64) take the stream-K path.
+SCHEDULE_CASES = [
+    # N, K, M, r
+    (2048, 1024, 300, 16),    # whole tiles: 32 FWD tiles of 16 K-steps
+    (2560, 256, 4000, 16),    # whole tiles: 320 FWD tiles, a ragged second wave
+    (4096, 512, 8, 16),       # stream-K: each tile cut between about five CTAs
+    (512, 4096, 64, 16),      # stream-K: 4 FWD tiles of 64 K-steps, ~37 CTAs per tile, more
+                              # partials than fit in shared memory
+    (1024, 256, 40, 32),      # stream-K: ragged token tile, 8 FWD / 2 DX tiles
+]
+
+
+@pytest.mark.parametrize("N,K,M,r", SCHEDULE_CASES)
+def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
+    """qlora_fused_fwd / qlora_fused_dx without a workspace (whole tiles per
+    CTA) and with one (stream-K, partial tiles summed through the workspace)
+    both match the oracle; the two differ only in fp32 summation order."""
+    import torch
+    s = 2.0
+    h, d = _setup(lib, N, K, M, r, index=5)
+    U = h["X"] @ h["A"].T
+    T = h["dY"] @ h["B"]
+    sU = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    sT = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    lws = torch.empty(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    lib.lora_xa(d["X"], d["A"], s, sU, lws)
+    lib.lora_dyb(d["dY"], d["B"], s, sT, lws)
+    gws = torch.full((lib.fused_workspace(M),), 0xAB, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = {}
+    for name, ws in (("whole", None), ("streamk", gws)):
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dX = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda")
+        lib.fused_fwd(d["q"], d["X"], d["B"], sU, Y, status=st, ws=ws)
+        lib.fused_dx(d["q"], d["dY"], d["A"], sT, dX, status=st, ws=ws)
+        out[name] = (Y, dX)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    Yr = olin.linear_fwd(h["Wd"], h["X"], h["A"], h["B"], s)[0]
+    dXr = h["dY"] @ h["Wd"] + s * (T @ h["A"])
+    for name, (Y, dX) in out.items():
+        assert_close_fp(bf16_dev_to_f64(Y), Yr, f"Y ({name})")
+        assert_close_fp(bf16_dev_to_f64(dX), dXr, f"dX ({name})")
+
+
+def test_stream_k_graph_replays(lib):
+    """A CUDA graph replays the stream-K forward with the same launch values
+    each time, so the flags in the workspace must be cleared by the kernel that
+    consumed them: three replays on changing inputs each match the oracle."""
+    import torch
+    N, K, M, r, s = 2048, 512, 40, 16, 2.0
+    h, d = _setup(lib, N, K, M, r, index=6)
+    sU = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    lws = torch.empty(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    gws = torch.empty(lib.fused_workspace(M), dtype=torch.uint8, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    X = d["X"].clone()
+    lib.lora_xa(X, d["A"], s, sU, lws)
+    lib.fused_fwd(d["q"], X, d["B"], sU, Y, ws=gws)    # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lib.lora_xa(X, d["A"], s, sU, lws)
+        lib.fused_fwd(d["q"], X, d["B"], sU, Y, ws=gws)
+    for rep in range(3):
+        c = inputs.linear_case(N, K, M, r, index=10 + rep)
+        X.copy_(to_dev_bf16(c["X"]))
+        Y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        Xh = inputs.bf16_bits_to_f32(c["X"]).astype(np.float64)
+        Yr = olin.linear_fwd(h["Wd"], Xh, h["A"], h["B"], s)[0]
+        assert_close_fp(bf16_dev_to_f64(Y), Yr, f"Y (replay {rep})")
+    del g
