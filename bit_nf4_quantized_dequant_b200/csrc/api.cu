@@ -211,6 +211,9 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   g.out = out;
   g.dev_status = dev_status;
   g.ws = ws;
+  if (mode == 0 && gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens: the weight-streaming kernel
+    return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, act, lora_w,
+                                           lora_act, r, out, reinterpret_cast<cudaStream_t>(stream)));
   return cuda_status(launch_fused_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 

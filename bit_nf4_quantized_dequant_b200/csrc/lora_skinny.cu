@@ -331,9 +331,10 @@ size_t cols_smem(int r_pad) {
 }
 
 // Cluster size for splitting a reduction of `blocks` 64-wide steps when
-// `tiles` CTAs already cover the output: enough CTAs to fill the GPU twice.
-int cluster_split(int64_t tiles, int64_t blocks) {
-  int64_t c = (2 * device_sm_count() + tiles - 1) / tiles;
+// `tiles` CTAs already cover the output: as many CTAs as are resident at once
+// (`per_sm` per SM, set by shared memory), never a second partial wave.
+int cluster_split(int64_t tiles, int64_t blocks, int per_sm) {
+  int64_t c = static_cast<int64_t>(per_sm) * device_sm_count() / tiles;
   if (c > kClusterMax) c = kClusterMax;
   if (c > blocks) c = blocks;
   if (c < 1) c = 1;
@@ -378,7 +379,7 @@ cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint
   if (!ok) return cudaErrorInvalidValue;
   const int64_t mtiles = (M + 63) / 64;
   const int64_t kblocks = (K + 63) / 64;
-  const int csize = cluster_split(mtiles, kblocks);
+  const int csize = cluster_split(mtiles, kblocks, static_cast<int>((228 * 1024) / (rows_smem(r_pad) + 1024)));
   int kb_per_cta = static_cast<int>((kblocks + csize - 1) / csize);
   int w_rk = w_is_rk ? 1 : 0;
   int32_t *status = nullptr;
@@ -410,7 +411,7 @@ cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, 
   const int tiles0 = static_cast<int>((K + 127) / 128);
   const int tiles1 = static_cast<int>((N + 127) / 128);
   const int64_t mblocks = (M + 63) / 64;
-  const int csize = cluster_split(tiles0 + tiles1, mblocks);
+  const int csize = cluster_split(tiles0 + tiles1, mblocks, static_cast<int>((228 * 1024) / (cols_smem(r_pad) + 1024)));
   int mb_per_cta = static_cast<int>((mblocks + csize - 1) / csize);
   ColsProblem p0{K, dA, 1}, p1{N, dB, 0};
   int t0v = tiles0;

@@ -36,6 +36,14 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t s);
 // Workspace of a stream-K launch with M tokens on the current device.
 size_t fused_gemm_ws_bytes(int64_t M);
 
+// Forward for M <= 16 tokens: dequantisation into warp-MMA register fragments,
+// K split over a thread-block cluster. Same result definition as the FWD mode
+// of the fused GEMM (fp32 accumulation, bf16 output).
+bool gemv_fwd_supported(int64_t N, int64_t K, int64_t M);
+cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, const float *scale2, int64_t N,
+                                int64_t K, int64_t M, const uint16_t *X, const uint16_t *Bl, const uint16_t *sU,
+                                int r, uint16_t *Y, cudaStream_t st);
+
 // Skinny LoRA products (fp32 accumulation).
 // out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if
 // w_is_rk else W[k*r + j].

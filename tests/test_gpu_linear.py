@@ -195,3 +195,26 @@ def test_stream_k_graph_replays(lib):
         Yr = olin.linear_fwd(h["Wd"], Xh, h["A"], h["B"], s)[0]
         assert_close_fp(bf16_dev_to_f64(Y), Yr, f"Y (replay {rep})")
     del g
+
+
+# Few-token forwards take the weight-streaming kernel (dequantisation into
+# warp-MMA register fragments, K split over a thread-block cluster).
+FEW_TOKEN_CASES = [
+    # N, K, M, r
+    (1024, 7168, 5, 16),    # cluster of 8, 14 NF4 blocks per CTA: a ragged last span
+    (512, 4096, 16, 32),    # two token tiles of 8
+    (2048, 1024, 9, 8),     # second token tile nearly empty
+    (64, 192, 3, 64),       # one row group, three blocks, largest rank
+]
+
+
+@pytest.mark.parametrize("N,K,M,r", FEW_TOKEN_CASES)
+def test_few_token_forward(lib, N, K, M, r):
+    import torch
+    s = 2.0
+    h, d = _setup(lib, N, K, M, r, index=7)
+    Y, sU = lib.linear_fwd(d["q"], d["X"], d["A"], d["B"], s)
+    torch.cuda.synchronize()
+    Yr, U = olin.linear_fwd(h["Wd"], h["X"], h["A"], h["B"], s)
+    assert_close_fp(bf16_dev_to_f64(sU), s * U, "sU")
+    assert_close_fp(bf16_dev_to_f64(Y), Yr, "Y")
