@@ -107,6 +107,20 @@ static qlora_status_t check_linear(const qlora_nf4_t *W, const uint16_t *X, int6
 
 static qlora_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
+// Forward for a few tokens in one launch (sU formed inside); validates like
+// qlora_linear_fwd apart from the workspace, which it does not use.
+qlora_status_t few_token_forward(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
+                                 qlora_stream_t stream) {
+  qlora_status_t st = check_linear(W, X, M, A, B, r, s);
+  if (st != QLORA_OK) return st;
+  if (!Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(Y) || (sU_out && !aligned16(sU_out))) return QLORA_ERR_MISALIGNED;
+  if (!gemv_fwd_supported(W->rows, W->cols, M)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, X, B, nullptr, A, s,
+                                         sU_out, r, Y, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -213,7 +227,8 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   g.ws = ws;
   if (mode == 0 && gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens: the weight-streaming kernel
     return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, act, lora_w,
-                                           lora_act, r, out, reinterpret_cast<cudaStream_t>(stream)));
+                                           lora_act, nullptr, 0.f, nullptr, r, out,
+                                           reinterpret_cast<cudaStream_t>(stream)));
   return cuda_status(launch_fused_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -254,6 +269,7 @@ qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   const WsLayout L = ws_layout(M, N, K, r);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  if (gemv_fwd_supported(N, K, M)) return few_token_forward(W, X, M, A, B, r, s, Y, sU_out, stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(wsb + L.su);
   st = qlora_lora_xa(X, M, K, A, r, s, sU, wsb + L.part, L.part_floats * 4, stream);

@@ -27,6 +27,15 @@
 //   partials through distributed shared memory in rank order, then adds the
 //   LoRA term in fp32 and stores bf16 (deterministic, no workspace).
 //
+// * Given the adapter A instead of sU, the kernel also computes the LoRA
+//   down-projection sU = bf16(s X A^T) itself. A cluster is cx row groups x cs
+//   K chunks; each CTA forms X A^T over its K chunk's spans congruent to its
+//   row-group index modulo cx (the same fragment scheme, A read from global
+//   memory in place of W', the activations already in shared memory), so a
+//   cluster reads A once; the partials are added over the whole cluster and
+//   rounded once; one CTA writes sU out for the backward. A few-token forward
+//   is then a single launch.
+//
 // CTA: 8 warps = 4 row tiles of 16 rows x 2 warps that split the CTA's spans.
 #include "qlora_device.cuh"
 
@@ -116,14 +125,19 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     nf4_gemv_fwd_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale8,
                         const float *__restrict__ scale2, int64_t N, int64_t K, int M,
                         const uint16_t *__restrict__ X, const uint16_t *__restrict__ Bl,
-                        const uint16_t *__restrict__ sU, int r, int blocks_per_cta, uint16_t *__restrict__ Y) {
+                        const uint16_t *__restrict__ sU, const uint16_t *__restrict__ Al, float s_lora,
+                        uint16_t *__restrict__ sU_out, int r, int blocks_per_cta, int cx,
+                        uint16_t *__restrict__ Y) {
   constexpr int mp = 8 * NTOK;
   constexpr uint32_t bstride = block_stride(mp);
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const uint32_t rank = cluster_ctarank();
+  // cluster = cx row groups (x) by csize K chunks (y); rank = x + y * cx
   const uint32_t csize = gridDim.y;
+  const uint32_t cxu = static_cast<uint32_t>(cx);
+  const uint32_t my_x = blockIdx.x % cxu;
+  const uint32_t rank = my_x + blockIdx.y * cxu;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
   const int64_t kblocks = K / 64;
   const int64_t cb0 = static_cast<int64_t>(blockIdx.y) * blocks_per_cta;
@@ -134,6 +148,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   uint8_t *xs = smem;                                                   // [4 * nspan blocks][mp][144 B]
   float *red = reinterpret_cast<float *>(smem + static_cast<size_t>(4 * nspan) * bstride);   // [2][64][mp]
   float *sum = red + 2 * kRowsPerCta * mp;                                                // [64][mp]
+  float *uslot = sum + kRowsPerCta * mp;   // [8 parts][64 j][mp]: X A^T partials of this CTA's warps
+  float *usum = uslot + 8 * 64 * mp;       // [64 j][mp]: this CTA's X A^T over its K range
+  float *su_s = usum + 64 * mp;            // [mp][64 j]: bf16(s X A^T) of all tokens, as float
 
   // Warp (rt, half) takes the spans half, half + 2, ... of its 16-row tile.
   // Its first three spans are requested before anything else so that their
@@ -163,10 +180,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
   __syncthreads();
 
+  const uint32_t xs_base = smem_u32(xs) + static_cast<uint32_t>(g * kTokStride + c * bstride);
   float d[NTOK][4];
 #pragma unroll
   for (int u = 0; u < NTOK; ++u) d[u][0] = d[u][1] = d[u][2] = d[u][3] = 0.f;
-  const uint32_t xs_base = smem_u32(xs) + static_cast<uint32_t>(g * kTokStride + c * bstride);
   for (int sp = half; sp < nsp; sp += 6) {
     compute_span<NTOK>(sa, d, xs_base + static_cast<uint32_t>(4 * sp) * bstride);
     load_span(sa, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 6, c);
@@ -176,6 +193,49 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     if (sp + 4 >= nsp) break;
     compute_span<NTOK>(sc, d, xs_base + static_cast<uint32_t>(4 * (sp + 4)) * bstride);
     load_span(sc, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 10, c);
+  }
+
+  const int jt_n = (r + 15) / 16;            // 16-row tiles of the adapter rank
+  if (Al != nullptr) {
+    // partial U[j, t] = sum over this CTA's K of A[j, k] X[t, k] (after the
+    // weight loop, when its registers are free): warp w takes
+    // rank tile w % jt_n and the spans congruent to w / jt_n modulo 8 / jt_n
+    const int parts = kWarps / jt_n;
+    if (warp < parts * jt_n) {
+      const int jt = warp % jt_n, part = warp / jt_n;
+      const int j0 = jt * 16 + g, j1 = j0 + 8;
+      float ud[NTOK][4];
+#pragma unroll
+      for (int u = 0; u < NTOK; ++u) ud[u][0] = ud[u][1] = ud[u][2] = ud[u][3] = 0.f;
+      for (int sp = static_cast<int>(my_x) + part * cx; sp < nspan; sp += parts * cx) {
+        const int lb = sp * 4 + c;
+        const bool valid = lb < nb_loc;
+        const uint16_t *a0 = Al + static_cast<int64_t>(j0) * K + (cb0 + lb) * 64;
+        const uint16_t *a1 = Al + static_cast<int64_t>(j1) * K + (cb0 + lb) * 64;
+        const uint32_t xrow = xs_base + static_cast<uint32_t>(4 * sp) * bstride;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 ra = valid && j0 < r ? __ldg(reinterpret_cast<const uint4 *>(a0 + 8 * i)) : make_uint4(0, 0, 0, 0);
+          const uint4 rb = valid && j1 < r ? __ldg(reinterpret_cast<const uint4 *>(a1 + 8 * i)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int u = 0; u < NTOK; ++u) {
+            const uint4 bx = lds_v4(xrow + static_cast<uint32_t>(u * 8 * kTokStride + i * 16));
+            const uint32_t a_lo[4] = {ra.x, rb.x, ra.y, rb.y};
+            const uint32_t a_hi[4] = {ra.z, rb.z, ra.w, rb.w};
+            mma_16816(ud[u], a_lo, bx.x, bx.y);
+            mma_16816(ud[u], a_hi, bx.z, bx.w);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < NTOK; ++u) {
+        float *dst = uslot + (part * 64 + jt * 16) * mp + 8 * u + 2 * c;
+        dst[g * mp] = ud[u][0];
+        dst[g * mp + 1] = ud[u][1];
+        dst[(g + 8) * mp] = ud[u][2];
+        dst[(g + 8) * mp + 1] = ud[u][3];
+      }
+    }
   }
 
   // ---- reduce: the two warps of a row tile, then the cluster's CTAs ----
@@ -190,11 +250,39 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kRowsPerCta * mp; i += blockDim.x) sum[i] = red[i] + red[kRowsPerCta * mp + i];
+  if (Al != nullptr) {
+    const int parts = kWarps / jt_n;
+    for (int i = threadIdx.x; i < jt_n * 16 * mp; i += blockDim.x) {
+      float u = 0.f;
+      for (int q = 0; q < parts; ++q) u += uslot[q * 64 * mp + i];
+      usum[i] = u;
+    }
+  }
   cluster_sync_all();
 
-  // rank q finishes rows [q * 64 / csize, (q + 1) * 64 / csize) of the CTA's 64
+  // the LoRA down-projection of all tokens, added over the cluster in rank order
+  if (Al != nullptr) {
+    const uint32_t usum_addr = smem_u32(usum);
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+      const int t = i / r, j = i % r;
+      const uint32_t off = static_cast<uint32_t>((j * mp + t) * 4);
+      float u = 0.f;
+      for (uint32_t q = 0; q < csize * cxu; ++q) u += ld_dsmem_f32(mapa_shared(usum_addr + off, q));
+      const __nv_bfloat16 v = __float2bfloat16_rn(s_lora * u);
+      su_s[t * 64 + j] = __bfloat162float(v);
+      if (sU_out != nullptr && blockIdx.x == 0 && rank == 0) sU_out[static_cast<int64_t>(t) * r + j] = __bfloat16_as_ushort(v);
+    }
+  } else {
+    for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+      const int t = i / r, j = i % r;
+      su_s[t * 64 + j] = __uint_as_float(static_cast<uint32_t>(sU[static_cast<int64_t>(t) * r + j]) << 16);
+    }
+  }
+  __syncthreads();
+
+  // K chunk q of a row group finishes rows [q * 64 / csize, (q + 1) * 64 / csize)
   const int rows_per = kRowsPerCta / static_cast<int>(csize);
-  const int rl0 = static_cast<int>(rank) * rows_per;
+  const int rl0 = static_cast<int>(blockIdx.y) * rows_per;
   const uint32_t sum_addr = smem_u32(sum);
   for (int i = threadIdx.x; i < rows_per * M; i += blockDim.x) {
     const int t = i / rows_per, rl = rl0 + i % rows_per;
@@ -202,12 +290,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     if (n >= N) continue;
     const uint32_t off = static_cast<uint32_t>((rl * mp + t) * 4);
     float y = 0.f;
-    for (uint32_t q = 0; q < csize; ++q) y += ld_dsmem_f32(mapa_shared(sum_addr + off, q));
+    for (uint32_t q = 0; q < csize; ++q) y += ld_dsmem_f32(mapa_shared(sum_addr + off, my_x + q * cxu));
     float l = 0.f;
     const uint16_t *brow = Bl + n * r;
-    const uint16_t *urow = sU + static_cast<int64_t>(t) * r;
-    for (int j = 0; j < r; ++j)
-      l = fmaf(__uint_as_float(static_cast<uint32_t>(urow[j]) << 16), __uint_as_float(static_cast<uint32_t>(brow[j]) << 16), l);
+    const float *urow = su_s + t * 64;
+    for (int j = 0; j < r; ++j) l = fmaf(urow[j], __uint_as_float(static_cast<uint32_t>(brow[j]) << 16), l);
     Y[static_cast<int64_t>(t) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y + l));
   }
   cluster_sync_all();   // no CTA leaves while another still reads its partials
@@ -220,7 +307,8 @@ size_t gemv_smem_bytes(int64_t K, int64_t M, int cs) {
   const int64_t kblocks = K / 64;
   const int64_t bpc = (kblocks + cs - 1) / cs;
   const int mp = M <= 8 ? 8 : 16;
-  return static_cast<size_t>(4 * ((bpc + 3) / 4)) * block_stride(mp) + static_cast<size_t>(3) * kRowsPerCta * mp * 4;
+  return static_cast<size_t>(4 * ((bpc + 3) / 4)) * block_stride(mp) +
+         static_cast<size_t>(3 * kRowsPerCta * mp + 8 * 64 * mp + 64 * mp + mp * 64) * 4;
 }
 
 // Cluster size (K split) for an [N, K] weight and M tokens, or 0 when the
@@ -244,10 +332,18 @@ bool gemv_fwd_supported(int64_t N, int64_t K, int64_t M) { return gemv_cluster(N
 
 cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, const float *scale2, int64_t N,
                                 int64_t K, int64_t M, const uint16_t *X, const uint16_t *Bl, const uint16_t *sU,
-                                int r, uint16_t *Y, cudaStream_t st) {
+                                const uint16_t *Al, float s, uint16_t *sU_out, int r, uint16_t *Y,
+                                cudaStream_t st) {
+  if ((sU == nullptr) == (Al == nullptr)) return cudaErrorInvalidValue;
   const int cs = gemv_cluster(N, K, M);
   if (cs == 0) return cudaErrorInvalidValue;
-  const int64_t row_groups = (N + kRowsPerCta - 1) / kRowsPerCta;
+  // with the adapter's down-projection inside, cx row groups share one
+  // cluster (and one read of A); the grid is padded to a multiple of cx
+  int cx = 1;
+  const int64_t rg_real = (N + kRowsPerCta - 1) / kRowsPerCta;
+  if (Al != nullptr)
+    while (cx * 2 * cs <= 8 && cx * 2 <= rg_real) cx *= 2;
+  const int64_t row_groups = (rg_real + cx - 1) / cx * cx;
   const int bpc = static_cast<int>((K / 64 + cs - 1) / cs);
   const int ntok = M <= 8 ? 1 : 2;
   const size_t smem = gemv_smem_bytes(K, M, cs);
@@ -262,13 +358,13 @@ cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, con
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cx);
   attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int Mi = static_cast<int>(M), bpc_arg = bpc;
-  void *args[] = {&codes, &scale8, &scale2, &N, &K, &Mi, &X, &Bl, &sU, &r, &bpc_arg, &Y};
+  void *args[] = {&codes, &scale8, &scale2, &N, &K, &Mi, &X, &Bl, &sU, &Al, &s, &sU_out, &r, &bpc_arg, &cx, &Y};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 

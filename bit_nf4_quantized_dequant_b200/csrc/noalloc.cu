@@ -62,6 +62,8 @@ extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const u
                                                    qlora_stream_t stream) {
   if (!W || !X || !A || !B || !Y || M <= 0 || W->rows <= 0 || W->cols <= 0) return QLORA_ERR_INVALID_ARG;
   if (W->cols % qlora::kBlock || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (qlora::gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens: one launch, no scratch at all
+    return qlora::few_token_forward(W, X, M, A, B, r, s, Y, sU_out, stream);
   // Scratch layout: [sU when the caller does not keep it][fp32 partial sums of s X A^T].
   const size_t su_bytes = sU_out ? 0 : round_up_256(static_cast<size_t>(M) * static_cast<size_t>(r) * 2);
   const size_t part_bytes = qlora::lora_rows_ws_floats(M, W->cols, r) * 4;

@@ -40,9 +40,22 @@ size_t fused_gemm_ws_bytes(int64_t M);
 // K split over a thread-block cluster. Same result definition as the FWD mode
 // of the fused GEMM (fp32 accumulation, bf16 output).
 bool gemv_fwd_supported(int64_t N, int64_t K, int64_t M);
+// Exactly one of sU (precomputed bf16(s X A^T)) and Al (the adapter A [r, K],
+// with s; the kernel then forms sU itself and writes it to sU_out if given).
 cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, const float *scale2, int64_t N,
                                 int64_t K, int64_t M, const uint16_t *X, const uint16_t *Bl, const uint16_t *sU,
-                                int r, uint16_t *Y, cudaStream_t st);
+                                const uint16_t *Al, float s, uint16_t *sU_out, int r, uint16_t *Y,
+                                cudaStream_t st);
+
+}  // namespace qlora
+
+#include "qlora.h"
+
+namespace qlora {
+// Few-token forward through the C-ABI types (validation + one launch).
+qlora_status_t few_token_forward(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
+                                 qlora_stream_t stream);
 
 // Skinny LoRA products (fp32 accumulation).
 // out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if

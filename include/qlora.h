@@ -113,7 +113,10 @@ qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r
  * W: NF4 weight [N, K] (struct on the host, buffers on the device).
  * X [M, K], A [r, K], B [N, r]: device bf16. Y [M, N]: device bf16, written.
  * sU_out [M, r]: device bf16 or NULL; if given, receives bf16_rn(s X A^T), the
- *   value the backward can reuse instead of recomputing it.
+ *   value the backward can reuse instead of recomputing it. For M <= 16 the
+ *   forward is a single launch that forms sU itself (its fp32 sum runs in a
+ *   different order than qlora_lora_xa's, so a backward that recomputes sU may
+ *   see it differ by bf16 rounding) and the workspace is not touched.
  * ws / ws_bytes: device workspace of at least qlora_linear_workspace() bytes.
  * dev_status: device int32 or NULL; set to QLORA_ERR_TIMEOUT if a bounded wait
  *   inside a kernel ran out (results are then incomplete). It is not cleared.

@@ -58,3 +58,25 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     rc = lib.library().qlora_linear_fwd_noalloc(ctypes.byref(q), P(0x40000), 1 << 22, P(0x50000), P(0x60000),
                                                 64, 2.0, P(0x70000), None, None, None)
     assert rc == 4   # QLORA_ERR_WORKSPACE
+
+
+def test_noalloc_few_tokens_needs_no_scratch(lib):
+    """At 12 tokens the forward is one launch that forms sU itself: the
+    allocation-free entry then touches no scratch at all, even for a K whose
+    partial sums would not fit in it, and matches the oracle."""
+    import numpy as np
+    import torch
+    from oracle import linear as olin, nf4 as onf4
+    N, K, M, r, s = 512, 4096, 12, 16, 2.0
+    c = inputs.linear_case(N, K, M, r, index=3)
+    q = lib.nf4_quantize(torch.from_numpy(c["W"]).cuda())
+    X, A, B = to_dev_bf16(c["X"]), to_dev_bf16(c["A"]), to_dev_bf16(c["B"])
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sU = torch.full((M, r), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _call_noalloc(lib, q, X, A, B, r, s, Y, sU) == 0
+    torch.cuda.synchronize()
+    Wd = onf4.dequantize(*onf4.quantize(c["W"]), N, K)
+    f = lambda b: inputs.bf16_bits_to_f32(b).astype(np.float64)
+    Yr, U = olin.linear_fwd(Wd, f(c["X"]), f(c["A"]), f(c["B"]), s)
+    assert_close_fp(bf16_dev_to_f64(Y), Yr, "Y")
+    assert_close_fp(bf16_dev_to_f64(sU), s * U, "sU")
