@@ -267,3 +267,62 @@ def dequantize_bits(packed: np.ndarray, scale8: np.ndarray, scale2: np.ndarray,
 def dequantize(packed, scale8, scale2, rows: int, cols: int) -> np.ndarray:
     """Dequantised weight as float64 values of the bf16 results."""
     return bf16_bits_to_f64(dequantize_bits(packed, scale8, scale2, rows, cols))
+
+
+# ---------------------------------------------------------------------------
+# Parts of a large matrix (for checks at full size that the oracle cannot
+# afford to encode whole). The block constants and the second-level groups
+# are computed over the whole matrix (a group of 256 blocks may straddle
+# rows); only the requested weights are encoded. The result equals the same
+# rows or columns of dequantize(*quantize(W)).
+# ---------------------------------------------------------------------------
+
+def _scales_all(W: np.ndarray):
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    c1 = block_absmax(W)
+    scale8, scale2 = double_quantize(c1)
+    return W, c1, block_scales(scale8, scale2).astype(np.float64), scale8, scale2
+
+
+def _dequant_blocks(Wb: np.ndarray, c1b: np.ndarray, sb: np.ndarray) -> np.ndarray:
+    """Blocks [nb, 64] of weights -> float64 values of their bf16 dequantisation."""
+    codes = encode_blocks(Wb, c1b, nf4_levels()).reshape(-1, BLOCK)
+    prod = (nf4_levels().astype(np.float64)[codes] * sb[:, None]).astype(np.float32)
+    return bf16_bits_to_f64(bf16_round_bits(prod.reshape(-1))).reshape(-1, BLOCK)
+
+
+def dequantize_rows(W: np.ndarray, rows) -> np.ndarray:
+    """Rows `rows` of the dequantised W (float64 [len(rows), K])."""
+    W, c1, s, _, _ = _scales_all(W)
+    N, K = W.shape
+    kb = K // BLOCK
+    rows = np.asarray(rows)
+    blocks = (rows[:, None] * kb + np.arange(kb)[None, :]).reshape(-1)
+    out = _dequant_blocks(W[rows].reshape(-1, BLOCK), c1[blocks], s[blocks])
+    return out.reshape(len(rows), K)
+
+
+def dequantize_cols(W: np.ndarray, cols) -> np.ndarray:
+    """Columns `cols` of the dequantised W (float64 [N, len(cols)])."""
+    W, c1, s, _, _ = _scales_all(W)
+    N, K = W.shape
+    kb = K // BLOCK
+    cols = np.asarray(cols)
+    cblocks = np.unique(cols // BLOCK)
+    blocks = (np.arange(N)[:, None] * kb + cblocks[None, :]).reshape(-1)
+    Wb = W.reshape(N, kb, BLOCK)[:, cblocks, :].reshape(-1, BLOCK)
+    vals = _dequant_blocks(Wb, c1[blocks], s[blocks]).reshape(N, len(cblocks), BLOCK)
+    where = np.searchsorted(cblocks, cols // BLOCK)
+    return vals[:, where, cols % BLOCK]
+
+
+def quantize_rows(W: np.ndarray, rows):
+    """(packed codes [len(rows), K/2], scale8 of those rows' blocks [len(rows), K/64],
+    scale2 of the whole matrix): the stored format restricted to `rows`."""
+    W, c1, _, scale8, scale2 = _scales_all(W)
+    N, K = W.shape
+    kb = K // BLOCK
+    rows = np.asarray(rows)
+    blocks = (rows[:, None] * kb + np.arange(kb)[None, :]).reshape(-1)
+    codes = encode_blocks(W[rows].reshape(-1, BLOCK), c1[blocks], nf4_levels())
+    return pack_codes(codes).reshape(len(rows), K // 2), scale8[blocks].reshape(len(rows), kb), scale2

@@ -226,3 +226,25 @@ def test_planted_tie_rule_is_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_midpoint_ties_go_to_lower_index()
     monkeypatch.setattr(nf4, "encode_blocks", real)
+
+
+@pytest.mark.parametrize("N,K", [(12, 11008), (12, 704), (33, 4096)])
+def test_row_and_column_restrictions_equal_the_whole(N, K):
+    """dequantize_rows / dequantize_cols / quantize_rows (used for checks at
+    full size) are the whole-matrix encoding restricted to rows or columns,
+    including second-level groups that straddle rows (K = 704 and 4096 give
+    11 and 64 blocks per row)."""
+    g = inputs.rng(31)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[3, 5] = 0.0
+    W[7, 64:128] = 0.0
+    packed, s8, s2 = nf4.quantize(W)
+    full = nf4.dequantize(packed, s8, s2, N, K)
+    rows = np.array([0, 3, 7, N - 1])
+    cols = np.array([0, 1, 63, 64, 65, K - 1, 130 if K > 130 else 2])
+    np.testing.assert_array_equal(nf4.dequantize_rows(W, rows), full[rows])
+    np.testing.assert_array_equal(nf4.dequantize_cols(W, cols), full[:, cols])
+    pr, s8r, s2r = nf4.quantize_rows(W, rows)
+    np.testing.assert_array_equal(pr, packed.reshape(N, K // 2)[rows])
+    np.testing.assert_array_equal(s8r, s8.reshape(N, K // 64)[rows])
+    np.testing.assert_array_equal(s2r, s2)
