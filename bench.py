@@ -230,6 +230,7 @@ def run_step(q, d, s, ev=None, side=None):
     main.wait_event(e_done)
 
 
+ALU_CLOCK_HZ = 1.965e9   # max SM clock of the machine's B200s (clocks.max.sm)
 LAUNCHES_PER_STEP = 5   # lora_xa, fused_fwd, lora_dyb, fused_dx, lora_grads: one kernel each
 
 
@@ -343,9 +344,19 @@ def bench_decode(q, torch, mats, steps, warmup):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     del graph
+    weights = sum(lin.N * lin.K for lin, _ in mats)
+    # The few-token forward is bound by the ALU pipe (table expansion), not HBM:
+    # 21 ALU operations per 8 weights plus 8 per 64-weight table; B200's ALU
+    # pipe retires 64 lanes per clock per SM.
+    alu_ops = weights * (21 / 8 + 8 / 64)
+    alu_peak = 64 * torch.cuda.get_device_properties(0).multi_processor_count * ALU_CLOCK_HZ
     return {"workload": "set_8b forward at 8 tokens: 224 matrices, r=16", "GB/s": moved / ms / 1e6,
             "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats),
-            "launch": "CUDA graph of the pass"}
+            "launch": "CUDA graph of the pass",
+            "roofline": {"kernel": "nf4_gemv_fwd_kernel", "bound": "alu", "achieved": alu_ops / (ms * 1e-3) / 1e12,
+                         "peak": alu_peak / 1e12, "unit": "T ALU lane-ops/s", "frac": alu_ops / (ms * 1e-3) / alu_peak,
+                         "ops_per_weight": 21 / 8 + 8 / 64,
+                         "peak_kind": "64 lanes/clk/SM x SMs x 1965 MHz (max SM clock)"}}
 
 
 # ---------------------------------------------------------------------------

@@ -58,6 +58,16 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
   return v;
 }
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros
+// (the global address is then not read).
+__device__ __forceinline__ void cp_async_16(uint32_t saddr, const void *gptr, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(gptr), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -153,9 +163,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   float *su_s = usum + 64 * mp;            // [mp][64 j]: bf16(s X A^T) of all tokens, as float
 
   // Warp (rt, half) takes the spans half, half + 2, ... of its 16-row tile.
-  // Its first three spans are requested before anything else so that their
-  // latency overlaps the activation fill; afterwards a span is requested as
-  // soon as its registers are consumed (three spans per warp in flight).
+  // Its first two spans are requested before anything else so that their
+  // latency overlaps the activation fill and the adapter projection; then a
+  // third; afterwards a span is requested as soon as its registers are
+  // consumed (three spans per warp in flight).
   const int rt = warp >> 1, half = warp & 1;
   const int64_t n0 = row0 + rt * 16 + g;
   const bool rows_ok = row0 + rt * 16 < N;   // N % 16 == 0: a row tile is all in or all out
@@ -163,42 +174,30 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
   SpanCodes sa, sb, sc;
   load_span(sa, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, half, c);
   load_span(sb, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, half + 2, c);
-  load_span(sc, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, half + 4, c);
 
-  // ---- activations of this K range -> shared memory (zero beyond M and K) ----
+  // ---- activations of this K range -> shared memory (zero beyond M and K),
+  // every 16-byte piece requested at once ----
   {
-    const int pieces = 4 * nspan * mp * 8;   // 16-byte pieces
+    const int pieces = 4 * nspan * mp * 8;
+    const uint32_t xs_s = smem_u32(xs);
     for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
       const int piece = i & 7;
       const int t = (i >> 3) % mp;
       const int lb = (i >> 3) / mp;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < M && lb < nb_loc)
-        v = *reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(t) * K + (cb0 + lb) * 64 + piece * 8);
-      *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(lb) * bstride + t * kTokStride + piece * 16) = v;
+      const bool in = t < M && lb < nb_loc;
+      const uint16_t *src = in ? X + static_cast<int64_t>(t) * K + (cb0 + lb) * 64 + piece * 8 : X;
+      cp_async_16(xs_s + static_cast<uint32_t>(lb) * bstride + static_cast<uint32_t>(t * kTokStride + piece * 16), src,
+                  in ? 16u : 0u);
     }
+    cp_async_wait_all();
   }
   __syncthreads();
 
   const uint32_t xs_base = smem_u32(xs) + static_cast<uint32_t>(g * kTokStride + c * bstride);
-  float d[NTOK][4];
-#pragma unroll
-  for (int u = 0; u < NTOK; ++u) d[u][0] = d[u][1] = d[u][2] = d[u][3] = 0.f;
-  for (int sp = half; sp < nsp; sp += 6) {
-    compute_span<NTOK>(sa, d, xs_base + static_cast<uint32_t>(4 * sp) * bstride);
-    load_span(sa, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 6, c);
-    if (sp + 2 >= nsp) break;
-    compute_span<NTOK>(sb, d, xs_base + static_cast<uint32_t>(4 * (sp + 2)) * bstride);
-    load_span(sb, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 8, c);
-    if (sp + 4 >= nsp) break;
-    compute_span<NTOK>(sc, d, xs_base + static_cast<uint32_t>(4 * (sp + 4)) * bstride);
-    load_span(sc, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 10, c);
-  }
-
   const int jt_n = (r + 15) / 16;            // 16-row tiles of the adapter rank
   if (Al != nullptr) {
-    // partial U[j, t] = sum over this CTA's K of A[j, k] X[t, k] (after the
-    // weight loop, when its registers are free): warp w takes
+    // partial U[j, t] = sum over this CTA's K of A[j, k] X[t, k], while the
+    // first weight spans are in flight: warp w takes
     // rank tile w % jt_n and the spans congruent to w / jt_n modulo 8 / jt_n
     const int parts = kWarps / jt_n;
     if (warp < parts * jt_n) {
@@ -236,6 +235,22 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
         dst[(g + 8) * mp + 1] = ud[u][3];
       }
     }
+  }
+
+  load_span(sc, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, half + 4, c);
+
+  float d[NTOK][4];
+#pragma unroll
+  for (int u = 0; u < NTOK; ++u) d[u][0] = d[u][1] = d[u][2] = d[u][3] = 0.f;
+  for (int sp = half; sp < nsp; sp += 6) {
+    compute_span<NTOK>(sa, d, xs_base + static_cast<uint32_t>(4 * sp) * bstride);
+    load_span(sa, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 6, c);
+    if (sp + 2 >= nsp) break;
+    compute_span<NTOK>(sb, d, xs_base + static_cast<uint32_t>(4 * (sp + 2)) * bstride);
+    load_span(sb, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 8, c);
+    if (sp + 4 >= nsp) break;
+    compute_span<NTOK>(sc, d, xs_base + static_cast<uint32_t>(4 * (sp + 4)) * bstride);
+    load_span(sc, codes, scale8, scale2, n0, K, cb0, nb_loc, nsp, sp + 10, c);
   }
 
   // ---- reduce: the two warps of a row tile, then the cluster's CTAs ----
