@@ -359,6 +359,84 @@ def bench_decode(q, torch, mats, steps, warmup):
                          "peak_kind": "64 lanes/clk/SM x SMs x 1965 MHz (max SM clock)"}}
 
 
+def bench_mlp_chain(q, torch, steps, warmup):
+    """Llama-7B SiLU-gated MLP (gate/up 4096->11008, down 11008->4096), 4096
+    tokens, r=16, alpha=32, one training step with gradient checkpointing:
+    forward, recompute of the layer's internals, backward (dX, dA, dB; no dW).
+    Two schedules of the same chain: three separate QLoRA linears with
+    silu(g) * u in torch between them, and the fused SwiGLU projection (gate
+    and up in one GEMM, h in its epilogue, g and u recomputed inside the
+    backward GEMM). Useful flops: 4 M N K per linear (fwd + dX)."""
+    import torch.nn.functional as Fn
+    H, F, M, r, s = 4096, 11008, 4096, 16, 2.0
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4242)
+    rnd = lambda *shape, std=1.0: torch.randn(*shape, generator=g, device="cuda") * std
+    Wg, Wu, Wd = rnd(F, H, std=0.02), rnd(F, H, std=0.02), rnd(H, F, std=0.02)
+    qg, qu, qd = q.nf4_quantize(Wg), q.nf4_quantize(Wu), q.nf4_quantize(Wd)
+    qgu = q.nf4_quantize(q.swiglu_interleave(Wg, Wu))
+    del Wg, Wu, Wd
+    bf = lambda t: t.bfloat16()
+    Ag, Au, Ad = bf(rnd(r, H, std=1 / r)), bf(rnd(r, H, std=1 / r)), bf(rnd(r, F, std=1 / r))
+    Bg, Bu, Bd = bf(rnd(F, r, std=0.01)), bf(rnd(F, r, std=0.01)), bf(rnd(H, r, std=0.01))
+    X, dY = bf(rnd(M, H)), bf(rnd(M, H))
+    Agu, Bgu = torch.cat([Ag, Au]), q.swiglu_pack_b(Bg, Bu)
+    ws_gu = torch.empty(q.linear_workspace(M, 2 * F, H, 2 * r), dtype=torch.uint8, device="cuda")
+    ws_g = torch.empty(q.linear_workspace(M, F, H, r), dtype=torch.uint8, device="cuda")
+    ws_d = torch.empty(q.linear_workspace(M, H, F, r), dtype=torch.uint8, device="cuda")
+    e = lambda *shape, dt=torch.bfloat16: torch.empty(*shape, dtype=dt, device="cuda")
+    b = dict(g=e(M, F), u=e(M, F), h=e(M, F), y=e(M, H), dh=e(M, F), dX=e(M, H), dXu=e(M, H),
+             sUg=e(M, r), sUu=e(M, r), sUd=e(M, r), sUgu=e(M, 2 * r), sTgu=e(M, 2 * r), dGU=e(M, 2 * F),
+             dAg=e(r, H, dt=torch.float32), dBg=e(F, r, dt=torch.float32), dAu=e(r, H, dt=torch.float32),
+             dBu=e(F, r, dt=torch.float32), dAd=e(r, F, dt=torch.float32), dBd=e(H, r, dt=torch.float32),
+             dAgu=e(2 * r, H, dt=torch.float32), dBgu=e(2 * F, 2 * r, dt=torch.float32))
+
+    def unfused():
+        for _ in range(2):   # forward, then the recompute before the backward
+            q.linear_fwd(qg, X, Ag, Bg, s, Y=b["g"], sU=b["sUg"], ws=ws_g)
+            q.linear_fwd(qu, X, Au, Bu, s, Y=b["u"], sU=b["sUu"], ws=ws_g)
+            torch.mul(Fn.silu(b["g"]), b["u"], out=b["h"])
+        q.linear_fwd(qd, b["h"], Ad, Bd, s, Y=b["y"], sU=b["sUd"], ws=ws_d)
+        q.linear_bwd(qd, b["h"], Ad, Bd, s, dY, sU=b["sUd"], dX=b["dh"], dA=b["dAd"], dB=b["dBd"], ws=ws_d)
+        gf, uf, dhf = b["g"].float(), b["u"].float(), b["dh"].float()
+        sig = torch.sigmoid(gf)
+        dg = (dhf * uf * sig * (1 + gf * (1 - sig))).bfloat16()
+        du = (dhf * Fn.silu(gf)).bfloat16()
+        q.linear_bwd(qg, X, Ag, Bg, s, dg, sU=b["sUg"], dX=b["dX"], dA=b["dAg"], dB=b["dBg"], ws=ws_g)
+        q.linear_bwd(qu, X, Au, Bu, s, du, sU=b["sUu"], dX=b["dXu"], dA=b["dAu"], dB=b["dBu"], ws=ws_g)
+        b["dX"].add_(b["dXu"])
+
+    def fused():
+        q.lora_xa(X, Agu, s, b["sUgu"], ws_gu)
+        q.swiglu_fwd(qgu, X, Bgu, b["sUgu"], H=b["h"])
+        q.linear_fwd(qd, b["h"], Ad, Bd, s, Y=b["y"], sU=b["sUd"], ws=ws_d)
+        q.swiglu_fwd(qgu, X, Bgu, b["sUgu"], H=b["h"])                   # recompute
+        q.linear_bwd(qd, b["h"], Ad, Bd, s, dY, sU=b["sUd"], dX=b["dh"], dA=b["dAd"], dB=b["dBd"], ws=ws_d)
+        q.swiglu_bwd(qgu, X, Bgu, b["sUgu"], b["dh"], dGU=b["dGU"])      # g, u recomputed inside
+        q.lora_dyb(b["dGU"], Bgu, s, b["sTgu"], ws_gu)
+        q.fused_dx(qgu, b["dGU"], Agu, b["sTgu"], b["dX"])
+        q.lora_grads(X, b["dGU"], b["sUgu"], b["sTgu"], b["dAgu"], b["dBgu"], ws_gu)
+        q.swiglu_unpack_db(b["dBgu"], b["dBg"], b["dBu"])
+
+    out = {"workload": "mlp_7b: gate/up 4096->11008, down 11008->4096, 4096 tokens, r=16, "
+                       "forward + recompute + backward"}
+    useful = 3 * 4 * M * F * H
+    for name, fn, executed in (("unfused", unfused, 3 * 6 * M * F * H), ("fused_swiglu", fused, 20 * M * F * H)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        out[name] = {"ms_per_step": ms, "useful_TFLOP/s": useful / (ms * 1e-3) / 1e12,
+                     "executed_TFLOP/s": executed / (ms * 1e-3) / 1e12}
+    return out
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (bounded sample)
 # ---------------------------------------------------------------------------
@@ -544,6 +622,8 @@ def main():
         extras["decode_fwd"] = bench_decode(q, torch, mats, steps=5, warmup=2)
         extras["decode_fwd"]["frac_of_hbm"] = extras["decode_fwd"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
         del mats
+        torch.cuda.empty_cache()
+        extras["mlp_chain"] = bench_mlp_chain(q, torch, steps=5, warmup=2)
     sampler.close()
 
     cpu = None

@@ -18,7 +18,7 @@ __all__ = [
     "nf4_sizes", "nf4_codebook", "nf4_quantize", "nf4_dequantize",
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
-    "fused_workspace",
+    "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +36,7 @@ SYMBOLS = [
     "qlora_linear_workspace", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_status_string",
     "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
     "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
+    "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
 ]
 
 
@@ -92,6 +93,14 @@ def library():
     lib.qlora_lora_xa.restype = st
     lib.qlora_lora_dyb.argtypes = [_P, _I64, _I64, _P, ctypes.c_int32, ctypes.c_float, _P, _P, _SZ, _P]
     lib.qlora_lora_dyb.restype = st
+    lib.qlora_swiglu_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P]
+    lib.qlora_swiglu_fwd.restype = st
+    lib.qlora_swiglu_bwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _P, _P]
+    lib.qlora_swiglu_bwd.restype = st
+    lib.qlora_swiglu_pack_b.argtypes = [_P, _P, _I64, ctypes.c_int32, _P, _P]
+    lib.qlora_swiglu_pack_b.restype = st
+    lib.qlora_swiglu_unpack_db.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
+    lib.qlora_swiglu_unpack_db.restype = st
     lib.qlora_fused_workspace.argtypes = [_I64, ctypes.POINTER(_SZ)]
     lib.qlora_fused_workspace.restype = st
     lib.qlora_fused_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P, _P]
@@ -304,3 +313,62 @@ def linear_fwd_noalloc(q: NF4Matrix, X, A, B, s: float, Y=None, sU=None, status=
     _check(library().qlora_linear_fwd_noalloc(ctypes.byref(st), _ptr(X), M, _ptr(A), _ptr(B), r, s, _ptr(Y),
                                               _ptr(sU), _ptr(status), _stream(stream)), "qlora_linear_fwd_noalloc")
     return Y, sU
+
+
+# ---------------------------------------------------------------------------
+# Fused SwiGLU projection (gate and up in one GEMM over the row-interleaved
+# weight; see include/qlora.h)
+# ---------------------------------------------------------------------------
+def swiglu_interleave(Wg, Wu):
+    """[Wg; Wu] with rows interleaved in chunks of 64 (a torch tensor op on the
+    float32 weights before quantisation; F % 64 == 0)."""
+    import torch
+    F, K = Wg.shape
+    return torch.stack([Wg.reshape(F // 64, 64, K), Wu.reshape(F // 64, 64, K)], 1).reshape(2 * F, K).contiguous()
+
+
+def swiglu_pack_b(Bg, Bu, out=None, stream=None):
+    """Block-diagonal [2F, 2r] up-projection of the fused product."""
+    import torch
+    F, r = Bg.shape
+    if out is None:
+        out = torch.empty((2 * F, 2 * r), dtype=torch.bfloat16, device=Bg.device)
+    _check(library().qlora_swiglu_pack_b(_ptr(Bg), _ptr(Bu), F, r, _ptr(out), _stream(stream)), "qlora_swiglu_pack_b")
+    return out
+
+
+def swiglu_unpack_db(dBgu, dBg=None, dBu=None, stream=None):
+    import torch
+    F2, r2 = dBgu.shape
+    F, r = F2 // 2, r2 // 2
+    if dBg is None:
+        dBg = torch.empty((F, r), dtype=torch.float32, device=dBgu.device)
+    if dBu is None:
+        dBu = torch.empty((F, r), dtype=torch.float32, device=dBgu.device)
+    _check(library().qlora_swiglu_unpack_db(_ptr(dBgu), F, r, _ptr(dBg), _ptr(dBu), _stream(stream)),
+           "qlora_swiglu_unpack_db")
+    return dBg, dBu
+
+
+def swiglu_fwd(q: NF4Matrix, X, Bgu, sUgu, H=None, status=None, stream=None):
+    """H = bf16(silu(g) u) for the interleaved gate/up weight q [2F, K]."""
+    import torch
+    M = X.shape[0]
+    if H is None:
+        H = torch.empty((M, q.rows // 2), dtype=torch.bfloat16, device=X.device)
+    st = q.c_struct()
+    _check(library().qlora_swiglu_fwd(ctypes.byref(st), _ptr(X), M, _ptr(Bgu), Bgu.shape[1], _ptr(sUgu), _ptr(H),
+                                      _ptr(status), _stream(stream)), "qlora_swiglu_fwd")
+    return H
+
+
+def swiglu_bwd(q: NF4Matrix, X, Bgu, sUgu, dH, dGU=None, status=None, stream=None):
+    """dGU [M, 2F] (dg in gate rows, du in up rows) with g, u recomputed."""
+    import torch
+    M = X.shape[0]
+    if dGU is None:
+        dGU = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    st = q.c_struct()
+    _check(library().qlora_swiglu_bwd(ctypes.byref(st), _ptr(X), M, _ptr(Bgu), Bgu.shape[1], _ptr(sUgu), _ptr(dH),
+                                      _ptr(dGU), _ptr(status), _stream(stream)), "qlora_swiglu_bwd")
+    return dGU

@@ -311,6 +311,69 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   return qlora_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, part, part_bytes, stream);
 }
 
+static qlora_status_t check_swiglu(const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M, const uint16_t *Bgu,
+                                   int32_t r2, const uint16_t *sUgu, const uint16_t *out) {
+  qlora_status_t st = check_linear(Wgu, X, M, Bgu, Bgu, r2, 1.0f);
+  if (st != QLORA_OK) return st;
+  if (!sUgu || !out) return QLORA_ERR_INVALID_ARG;
+  if (Wgu->rows % 128 || r2 % 2) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(sUgu) || !aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+static qlora_status_t swiglu_launch(int mode, const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M,
+                                   const uint16_t *Bgu, int32_t r2, const uint16_t *sUgu, const uint16_t *dH,
+                                   uint16_t *out, int32_t *dev_status, qlora_stream_t stream) {
+  GemmArgs g{};
+  g.mode = mode;
+  g.codes = Wgu->codes;
+  g.scale8 = Wgu->scale8;
+  g.scale2 = Wgu->scale2;
+  g.N = Wgu->rows;
+  g.K = Wgu->cols;
+  g.M = M;
+  g.r = r2;
+  g.act = X;
+  g.lora_w = Bgu;
+  g.lora_act = sUgu;
+  g.out = out;
+  g.dev_status = dev_status;
+  g.aux = dH;
+  return cuda_status(launch_fused_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_swiglu_fwd(const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M, const uint16_t *Bgu,
+                                int32_t r2, const uint16_t *sUgu, uint16_t *H, int32_t *dev_status,
+                                qlora_stream_t stream) {
+  qlora_status_t st = check_swiglu(Wgu, X, M, Bgu, r2, sUgu, H);
+  if (st != QLORA_OK) return st;
+  return swiglu_launch(2, Wgu, X, M, Bgu, r2, sUgu, nullptr, H, dev_status, stream);
+}
+
+qlora_status_t qlora_swiglu_bwd(const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M, const uint16_t *Bgu,
+                                int32_t r2, const uint16_t *sUgu, const uint16_t *dH, uint16_t *dGU,
+                                int32_t *dev_status, qlora_stream_t stream) {
+  qlora_status_t st = check_swiglu(Wgu, X, M, Bgu, r2, sUgu, dGU);
+  if (st != QLORA_OK) return st;
+  if (!dH) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dH)) return QLORA_ERR_MISALIGNED;
+  return swiglu_launch(3, Wgu, X, M, Bgu, r2, sUgu, dH, dGU, dev_status, stream);
+}
+
+qlora_status_t qlora_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t F, int32_t r, uint16_t *Bgu,
+                                   qlora_stream_t stream) {
+  if (!Bg || !Bu || !Bgu || F <= 0) return QLORA_ERR_INVALID_ARG;
+  if (F % 64 || r < 4 || r > 32 || r % 4) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return cuda_status(launch_swiglu_pack_b(Bg, Bu, F, r, Bgu, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status_t qlora_swiglu_unpack_db(const float *dBgu, int64_t F, int32_t r, float *dBg, float *dBu,
+                                      qlora_stream_t stream) {
+  if (!dBgu || !dBg || !dBu || F <= 0) return QLORA_ERR_INVALID_ARG;
+  if (F % 64 || r < 4 || r > 32 || r % 4) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return cuda_status(launch_swiglu_unpack_db(dBgu, F, r, dBg, dBu, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *qlora_status_string(qlora_status_t status) {
   switch (status) {
     case QLORA_OK: return "QLORA_OK";

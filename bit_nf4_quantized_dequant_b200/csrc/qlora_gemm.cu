@@ -64,7 +64,7 @@ struct GemmParams {
   const float *scale2;
   int32_t *status;
   int64_t N, K, M;
-  int mode;        // 0 FWD, 1 DX
+  int mode;        // 0 FWD, 1 DX, 2 SwiGLU FWD (h), 3 SwiGLU BWD (dg, du); 2 and 3 run the FWD main loop
   int bt;          // token tile of one (pair) tile = UMMA N
   int bt_cta;      // tokens whose activations this CTA loads (bt, or bt / 2 for a pair)
   int sx, sa, sc;  // ring depths: activations, dequantised tiles, codes
@@ -97,7 +97,7 @@ __device__ __forceinline__ uint32_t lora_layout(int r_pad) {
 struct Smem {
   uint8_t *x, *a, *lb, *la, *out, *c;
   uint32_t x_bytes;
-  uint64_t *xf, *xe, *af, *ae, *cf, *ce, *lf, *le, *accf, *acce, *drain, *peer_full;
+  uint64_t *xf, *xe, *af, *ae, *cf, *ce, *lf, *le, *accf, *acce, *drain, *peer_full, *dhf;
   uint32_t *tmem_holder;
   int *abort_flag;
 };
@@ -120,7 +120,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmParams &p) {
   s.accf = s.le + 1;  s.acce = s.accf + 2;
   s.drain = s.acce + 2;
   s.peer_full = s.drain + 1;
-  s.tmem_holder = reinterpret_cast<uint32_t *>(s.peer_full + 1);
+  s.dhf = s.peer_full + 1;
+  s.tmem_holder = reinterpret_cast<uint32_t *>(s.dhf + 2);
   s.abort_flag = reinterpret_cast<int *>(s.tmem_holder + 1);
   return s;
 }
@@ -189,13 +190,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_codes,
                           const __grid_constant__ CUtensorMap tm_lora_w,
                           const __grid_constant__ CUtensorMap tm_lora_act,
-                          const __grid_constant__ CUtensorMap tm_out, const GemmParams p) {
+                          const __grid_constant__ CUtensorMap tm_out,
+                          const __grid_constant__ CUtensorMap tm_aux,   // dH (mode 3), else unused
+                          const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Smem sm = carve(base, p);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool dx = p.mode == 1;
+  const bool swiglu = p.mode >= 2;
   // CTA pair: rank 0 (even CTA) issues the MMAs; rank 1 is its peer.
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
@@ -238,6 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) { mbar_init(&sm.accf[i], 1); mbar_init(&sm.acce[i], per_step); }
     mbar_init(sm.drain, 1);
     mbar_init(sm.peer_full, 1);
+    mbar_init(&sm.dhf[0], 1);
+    mbar_init(&sm.dhf[1], 1);
     *sm.abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -247,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_lora_w);
     tma_prefetch_desc(&tm_lora_act);
     tma_prefetch_desc(&tm_out);
+    if (p.mode == 3) tma_prefetch_desc(&tm_aux);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -439,6 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int box_t = p.bt < kEpiTokens ? p.bt : kEpiTokens;
     const int nchunks = p.bt / box_t;
     uint32_t chunk_count = 0;
+    uint32_t dh_count = 0;   // dH chunk loads so far (SwiGLU backward): buffer and phase
     StepPos seg;
     seg.init(walk);
     const int64_t part_elems = static_cast<int64_t>(kTileRows) * p.bt;
@@ -490,6 +498,103 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_release_gpu_u64(p.flags + blockIdx.x, p.epoch);
         }
         __syncwarp();
+      } else if (swiglu) {
+        // SwiGLU tile: weight rows 0..63 are gate rows and 64..127 the up rows
+        // of the same 64 output columns (the weight is [Wg; Wu] interleaved in
+        // 64-row chunks), so TMEM lanes 0..63 hold g and lanes 64..127 hold u
+        // for the tile's tokens. g and u are rounded to bf16 (the compute dtype
+        // of the layer outputs) and exchanged between the two halves through
+        // shared memory, 32 tokens at a time.
+        const bool gate = q < 2;
+        const int hr = et & 63;
+        const uint32_t dh_bytes = static_cast<uint32_t>(box_t) * 64u * 2u;
+        auto dh_buf = [&](uint32_t k) {
+          return reinterpret_cast<uint16_t *>(sm.out + kOutStageBytes + (k & 1u) * (kOutStageBytes / 2));
+        };
+        if (p.mode == 3 && et == 0) {   // dH for the first 32 tokens of the tile
+          mbar_arrive_expect_tx(&sm.dhf[dh_count & 1u], dh_bytes);
+          tma_load_2d(dh_buf(dh_count), &tm_aux, &sm.dhf[dh_count & 1u], rt * 64, tt * p.bt);
+        }
+        for (int c = 0; c < nchunks; ++c, ++chunk_count) {
+          uint32_t v[32];
+          tmem_ld32(taddr + static_cast<uint32_t>(c * box_t), v);
+          tmem_ld_wait();
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_leader(&sm.acce[buf]);
+          }
+          if (p.mode == 2) {
+            // h = bf16(silu(g) * u) -> H[tokens, 64 columns]
+            uint8_t *cb = sm.out + (chunk_count & 1u) * kOutStageBytes;
+            uint16_t *ux = reinterpret_cast<uint16_t *>(cb);          // [32 tokens][64] u
+            uint16_t *hs = reinterpret_cast<uint16_t *>(cb + 4096);   // [32 tokens][64] h
+            if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
+            named_barrier(1, 128);
+            if (!gate) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < box_t) ux[j * 64 + hr] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            }
+            named_barrier(1, 128);
+            if (gate) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < box_t) {
+                  const float g = __bfloat162float(__float2bfloat16_rn(__uint_as_float(v[j])));
+                  const float u = __uint_as_float(static_cast<uint32_t>(ux[j * 64 + hr]) << 16);
+                  const float h = __fdividef(g, 1.f + __expf(-g)) * u;
+                  hs[j * 64 + hr] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                }
+              }
+            }
+            fence_proxy_async_smem();
+            named_barrier(1, 128);
+            if (et == 0) {
+              tma_store_2d(&tm_out, hs, rt * 64, tt * p.bt + c * box_t);
+              bulk_commit_group();
+            }
+          } else {
+            // dg = dh * u * silu'(g), du = dh * silu(g) -> dGU[tokens, 128 rows]
+            uint16_t *xch = reinterpret_cast<uint16_t *>(sm.out);   // [32 tokens][128] g | u, then dg | du
+            if (c + 1 < nchunks && et == 0) {   // dH of the next 32 tokens into the other buffer
+              const uint32_t k = dh_count + 1;
+              mbar_arrive_expect_tx(&sm.dhf[k & 1u], dh_bytes);
+              tma_load_2d(dh_buf(k), &tm_aux, &sm.dhf[k & 1u], rt * 64, tt * p.bt + (c + 1) * box_t);
+            }
+            if (et == 0) bulk_wait_group_read<0>();   // the previous store has read the buffer
+            named_barrier(1, 128);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < box_t) xch[j * 128 + et] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            mbar_wait(&sm.dhf[dh_count & 1u], (dh_count >> 1) & 1u, abort_flag, p.status);
+            named_barrier(1, 128);
+            const uint16_t *dhb = dh_buf(dh_count);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < box_t) {
+                const float own = __uint_as_float(static_cast<uint32_t>(xch[j * 128 + et]) << 16);
+                const float other = __uint_as_float(static_cast<uint32_t>(xch[j * 128 + (et ^ 64)]) << 16);
+                const float g = gate ? own : other, u = gate ? other : own;
+                const float d = __uint_as_float(static_cast<uint32_t>(dhb[j * 64 + hr]) << 16);
+                const float sg = __frcp_rn(1.f + __expf(-g));
+                v[j] = __float_as_uint(gate ? d * u * sg * (1.f + g * (1.f - sg)) : d * g * sg);
+              }
+            }
+            named_barrier(1, 128);   // every exchange read is done
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < box_t) xch[j * 128 + et] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            fence_proxy_async_smem();
+            named_barrier(1, 128);
+            if (et == 0) {
+              tma_store_2d(&tm_out, xch, rt * kTileRows, tt * p.bt + c * box_t);
+              bulk_commit_group();
+            }
+            ++dh_count;
+          }
+          __syncwarp();
+        }
       } else {
         // tail: CTAs blockIdx.x + 1 .. blockIdx.x + n_peers hold the rest of this tile
         int n_peers = 0, n_smem = 0;
@@ -686,7 +791,7 @@ size_t smem_bytes(int bt_cta, int r_pad, int sx, int sa, int sc) {
   return 1024 /* alignment slack */ + static_cast<size_t>(sx) * bt_cta * 128u +
          static_cast<size_t>(sa) * kATileBytes + lora_b_bytes(bt_cta, r_pad) + lora_a_bytes(r_pad) +
          2 * kOutStageBytes + static_cast<size_t>(sc) * kCodeTileBytes +
-         static_cast<size_t>(2 * (sx + sa + sc) + 8) * 8 + 16;
+         static_cast<size_t>(2 * (sx + sa + sc) + 10) * 8 + 16;
 }
 
 // Ring depths that fit the shared-memory budget, in order of preference: at
@@ -749,26 +854,30 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   p.bt_cta = pair ? bt / 2 : bt;
   p.r_pad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
   pick_rings(p.bt_cta, p.r_pad, p.sx, p.sa, p.sc);
-  const int64_t rows = a.mode == 0 ? a.N : a.K;         // weight extent along UMMA M
+  const int64_t rows = a.mode == 1 ? a.K : a.N;         // weight extent along UMMA M
   const int rows_per_tile = pair ? 2 * kTileRows : kTileRows;
   p.row_tiles = static_cast<int>((rows + rows_per_tile - 1) / rows_per_tile);
   p.tok_tiles = static_cast<int>((a.M + bt - 1) / bt);
-  p.nk = static_cast<int>(a.mode == 0 ? a.K / kKStage : (a.N + kKStage - 1) / kKStage);
+  p.nk = static_cast<int>(a.mode != 1 ? a.K / kKStage : (a.N + kKStage - 1) / kKStage);
 
-  CUtensorMap tm_act, tm_codes, tm_lw, tm_la, tm_out;
+  CUtensorMap tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux;
   const CUtensorMapSwizzle lsw = lora_swizzle(p.r_pad);
   const uint32_t box_t = bt < kEpiTokens ? bt : kEpiTokens;
   const uint32_t bt_cta = static_cast<uint32_t>(p.bt_cta);
   bool ok = true;
-  if (a.mode == 0) {
+  if (a.mode != 1) {
     ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.K, a.M, a.K * 2, 64, bt_cta,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= encode_2d(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, a.K / 2, a.N, a.K / 2, 32,
                     kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE);
     ok &= encode_2d(&tm_lw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lora_w, a.r, a.N, a.r * 2, p.r_pad,
                     kTileRows, lsw);
-    ok &= encode_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.N * 2, kTileRows,
-                    box_t, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (a.mode == 2)   // H [M, N / 2], 64 columns per tile
+      ok &= encode_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N / 2, a.M, a.N, 64, box_t,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+      ok &= encode_2d(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.N * 2, kTileRows,
+                      box_t, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
     ok &= encode_2d(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.act, a.N, a.M, a.N * 2, 64, bt_cta,
                     CU_TENSOR_MAP_SWIZZLE_128B);
@@ -781,6 +890,11 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   }
   ok &= encode_2d(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lora_act, a.r, a.M, a.r * 2, p.r_pad,
                   bt_cta, lsw);
+  if (a.mode == 3)   // dH [M, N / 2]
+    ok &= encode_2d(&tm_aux, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.aux, a.N / 2, a.M, a.N, 64, box_t,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    tm_aux = tm_out;
   if (!ok) return cudaErrorInvalidValue;
 
   const size_t smem = smem_bytes(p.bt_cta, p.r_pad, p.sx, p.sa, p.sc);
@@ -791,7 +905,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     int grid = ntiles < sms ? ntiles : sms;
-    if (a.ws && bt <= 64) {
+    if (a.ws && bt <= 64 && a.mode <= 1) {
       // Stream-K over all SMs for short token tiles: a few weight-row tiles
       // would otherwise occupy a few SMs, and the fp32 partials that cross
       // CTAs are small. With 128- and 256-token tiles the partials (64 and
@@ -805,7 +919,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
       p.flags = static_cast<uint64_t *>(a.ws);
       p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + flags);
     }
-    fused_nf4_gemm_kernel<false><<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, p);
+    fused_nf4_gemm_kernel<false><<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux, p);
     return cudaGetLastError();
   }
   cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -824,7 +938,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void *args[] = {&tm_act, &tm_codes, &tm_lw, &tm_la, &tm_out, &p};
+  void *args[] = {&tm_act, &tm_codes, &tm_lw, &tm_la, &tm_out, &tm_aux, &p};
   return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true>), args);
 }
 

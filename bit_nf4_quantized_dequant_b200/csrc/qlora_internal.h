@@ -18,8 +18,11 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const
 
 // Fused NF4 GEMM (tcgen05). Mode FWD: Y[M,N] = X[M,K] W'^T + sU[M,r] Bl^T.
 // Mode DX: dX[M,K] = dY[M,N] W' + sT[M,r] Al.
+// SwiGLU modes (W = [Wg; Wu] interleaved in 64-row chunks, N = 2F): the FWD
+// product G|U, then 2: out = H[M,F] = bf16(silu(g) u); 3: out = dGU[M,N] with
+// dg = dH u silu'(g) in gate rows and du = dH silu(g) in up rows (aux = dH[M,F]).
 struct GemmArgs {
-  int mode;                 // 0 = FWD, 1 = DX
+  int mode;                 // 0 = FWD, 1 = DX, 2 = SwiGLU FWD, 3 = SwiGLU BWD
   const uint8_t *codes;
   const uint8_t *scale8;
   const float *scale2;
@@ -31,6 +34,7 @@ struct GemmArgs {
   uint16_t *out;            // Y [M, N] or dX [M, K]
   int32_t *dev_status;
   void *ws;                 // optional stream-K workspace (fused_gemm_ws_bytes(M) bytes), or null
+  const uint16_t *aux;      // dH [M, N/2] for mode 3
 };
 cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t s);
 // Workspace of a stream-K launch with M tokens on the current device.
@@ -52,6 +56,11 @@ cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, con
 #include "qlora.h"
 
 namespace qlora {
+// SwiGLU layout helpers (see swiglu_pack.cu).
+cudaError_t launch_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t F, int r, uint16_t *Bgu,
+                                 cudaStream_t st);
+cudaError_t launch_swiglu_unpack_db(const float *dBgu, int64_t F, int r, float *dBg, float *dBu, cudaStream_t st);
+
 // Few-token forward through the C-ABI types (validation + one launch).
 qlora_status_t few_token_forward(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
                                  const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,

@@ -206,6 +206,51 @@ qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M
                                 void *ws, size_t ws_bytes, qlora_stream_t stream);
 
 /*
+ * Fused SwiGLU projection of the Llama-style MLP, h = silu(g) * u with
+ * g = X Wg'^T + sU_g B_g^T and u = X Wu'^T + sU_u B_u^T ("QLoRA and Fine-Tuning
+ * on One Consumer GPU", section "Where 24 GB goes": adapters on the MLP
+ * projections, and gradient checkpointing recomputes a layer's MLP
+ * intermediates during the backward). The pages do not define this fusion;
+ * it is a kernel of this library that computes the same chain as the separate
+ * linears with g and u rounded to bf16 before silu, as the unfused chain does.
+ *
+ * Layout: Wgu is the NF4 quantisation of [Wg; Wu] with rows interleaved in
+ * chunks of 64 (rows 128c..128c+63 = gate rows 64c.., rows 128c+64.. = up rows
+ * 64c..), [2F, K] with F % 64 == 0 and K % 64 == 0. Bgu [2F, 2r] bf16 is the
+ * block-diagonal up-projection in the same row order (qlora_swiglu_pack_b);
+ * sUgu [M, 2r] = [sU_g | sU_u], e.g. qlora_lora_xa with A_gu = [A_g; A_u]
+ * [2r, K]. r2 = 2r with 8 <= r2 <= 64, r2 % 8 == 0.
+ */
+
+/* H [M, F] bf16 = bf16(silu(bf16(g)) * bf16(u)) in one tcgen05 GEMM over Wgu.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+qlora_status_t qlora_swiglu_fwd(const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M, const uint16_t *Bgu,
+                                int32_t r2, const uint16_t *sUgu, uint16_t *H, int32_t *dev_status,
+                                qlora_stream_t stream);
+
+/* Backward through silu(g) * u with g and u recomputed inside the GEMM (they
+ * are never stored): dGU [M, 2F] bf16 in Wgu's row order, dg = dH u silu'(g)
+ * in gate rows and du = dH silu(g) in up rows (g, u as in qlora_swiglu_fwd).
+ * dX then follows from qlora_fused_dx over Wgu with A_gu and sT_gu =
+ * qlora_lora_dyb(dGU, Bgu); qlora_lora_grads(X, dGU, sUgu, sTgu) gives
+ * [dA_g; dA_u] and a [2F, 2r] dB whose diagonal blocks are dB_g, dB_u
+ * (qlora_swiglu_unpack_db). dH [M, F] bf16. Errors: as qlora_swiglu_fwd. */
+qlora_status_t qlora_swiglu_bwd(const qlora_nf4_t *Wgu, const uint16_t *X, int64_t M, const uint16_t *Bgu,
+                                int32_t r2, const uint16_t *sUgu, const uint16_t *dH, uint16_t *dGU,
+                                int32_t *dev_status, qlora_stream_t stream);
+
+/* Bgu [2F, 2r] from B_g, B_u [F, r] (device bf16): gate row [B_g row | 0],
+ * up row [0 | B_u row], rows interleaved as in Wgu. F % 64 == 0, 4 <= r <= 32,
+ * r % 4 == 0. Errors: INVALID_ARG, UNSUPPORTED_SHAPE, CUDA. */
+qlora_status_t qlora_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t F, int32_t r, uint16_t *Bgu,
+                                   qlora_stream_t stream);
+
+/* dB_g, dB_u [F, r] fp32 from the diagonal blocks of dBgu [2F, 2r] fp32.
+ * Errors: as qlora_swiglu_pack_b. */
+qlora_status_t qlora_swiglu_unpack_db(const float *dBgu, int64_t F, int32_t r, float *dBg, float *dBu,
+                                      qlora_stream_t stream);
+
+/*
  * Allocation-free forward. The pages have no counterpart to this call: it is an
  * interface convenience of this library for callers that cannot allocate
  * device memory where they run the layer (a plug-in that only receives its

@@ -123,25 +123,52 @@ def test_set_8b_dequant_bit_exact_on_sampled_rows(lib, N, K):
     np.testing.assert_array_equal(bf16_dev_bits(Wd)[rows], ref_bits)
 
 
-def test_mlp_7b_chain_with_recompute(lib):
-    """Llama-7B SiLU-gated MLP (gate/up 4096->11008, down 11008->4096), 4096
-    tokens, r=16, alpha=32, with the gradient-checkpointing pattern: the
-    forward runs, is recomputed (dequantising every weight again) and must
-    give the same bits, then the backward runs through SiLU(g) * u. The glue
-    between the layers is plain torch in bf16; the oracle follows the same
-    chain in float64, rounding to bf16 at the same layer boundaries."""
-    import torch
-    import torch.nn.functional as F
+@pytest.fixture(scope="module")
+def mlp_7b():
+    """Inputs and the float64 oracle of the Llama-7B SiLU-gated MLP chain
+    (gate/up 4096->11008, down 11008->4096), 4096 tokens, r=16, alpha=32,
+    computed once for the unfused and the fused chain. The oracle rounds to
+    bf16 at the layer boundaries the kernels round at (g, u, h, dH, dg, du)."""
     H, Fd, M, r, alpha = 4096, 11008, 4096, 16, 32.0
     s = alpha / r
+
     def case(N, K, index):   # only the inputs the chain uses
         return dict(W=inputs.weight_f32(N, K, index), A=inputs.lora_a_bf16(r, K, index),
                     B=inputs.lora_b_bf16(N, r, index))
     cg, cu, cd = case(Fd, H, 80), case(Fd, H, 81), case(H, Fd, 82)
-    cg["X"] = inputs.activations_bf16(M, H, 80)
-    cd["dY"] = inputs.grad_out_bf16(M, H, 82)
-    X = to_dev_bf16(cg["X"])
-    dY = to_dev_bf16(cd["dY"])
+    X, dY = inputs.activations_bf16(M, H, 80), inputs.grad_out_bf16(M, H, 82)
+    Wg, Wu, Wd = (onf4.dequantize(*onf4.quantize(c["W"]), *c["W"].shape) for c in (cg, cu, cd))
+    Xh, dYh = _f64(X), _f64(dY)
+    (Ag, Bg), (Au, Bu), (Ad, Bd) = ((_f64(c["A"]), _f64(c["B"])) for c in (cg, cu, cd))
+    go = _bf16r(olin.linear_fwd(Wg, Xh, Ag, Bg, s)[0])
+    uo = _bf16r(olin.linear_fwd(Wu, Xh, Au, Bu, s)[0])
+    silu = go / (1.0 + np.exp(-go))
+    ho = _bf16r(silu * uo)
+    yo = olin.linear_fwd(Wd, ho, Ad, Bd, s)[0]
+    dho, dAdo, dBdo = olin.linear_bwd(Wd, ho, Ad, Bd, s, dYh)
+    dho = _bf16r(dho)
+    sg = 1.0 / (1.0 + np.exp(-go))
+    dgo = _bf16r(dho * uo * sg * (1 + go * (1 - sg)))
+    duo = _bf16r(dho * silu)
+    dXgo, dAgo, dBgo = olin.linear_bwd(Wg, Xh, Ag, Bg, s, dgo)
+    dXuo, dAuo, dBuo = olin.linear_bwd(Wu, Xh, Au, Bu, s, duo)
+    return dict(s=s, r=r, cg=cg, cu=cu, cd=cd, X=X, dY=dY,
+                ref=dict(g=go, h=ho, y=yo, dh=dho, dX=dXgo + dXuo, dAd=dAdo, dBd=dBdo, dAg=dAgo, dBg=dBgo,
+                         dAu=dAuo, dBu=dBuo))
+
+
+def test_mlp_7b_chain_with_recompute(lib, mlp_7b):
+    """The chain through three separate QLoRA linears with the
+    gradient-checkpointing pattern: the forward runs, is recomputed
+    (dequantising every weight again) and must give the same bits, then the
+    backward runs through SiLU(g) * u. The glue between the layers is plain
+    torch in bf16."""
+    import torch
+    import torch.nn.functional as F
+    d, s = mlp_7b, mlp_7b["s"]
+    cg, cu, cd = d["cg"], d["cu"], d["cd"]
+    X = to_dev_bf16(d["X"])
+    dY = to_dev_bf16(d["dY"])
     qs, lora = [], []
     for c in (cg, cu, cd):
         qs.append(lib.nf4_quantize(torch.from_numpy(c["W"]).cuda()))
@@ -168,29 +195,59 @@ def test_mlp_7b_chain_with_recompute(lib):
     dXu, dAu, dBu = lib.linear_bwd(qs[1], X, *lora[1], s, du, sU=sUs[1])
     dX = dXg.float() + dXu.float()
     torch.cuda.synchronize()
+    ref = d["ref"]
+    assert_close_fp(bf16_dev_to_f64(g), ref["g"], "gate output")
+    assert_close_fp(bf16_dev_to_f64(h), ref["h"], "SiLU(g) * u")
+    assert_close_fp(bf16_dev_to_f64(y), ref["y"], "MLP output")
+    assert_close_fp(bf16_dev_to_f64(dh), ref["dh"], "dH")
+    assert_close_fp(dX.double().cpu().numpy(), ref["dX"], "dX")
+    for name, got in (("dAd", dAd), ("dBd", dBd), ("dAg", dAg), ("dBg", dBg), ("dAu", dAu), ("dBu", dBu)):
+        assert_close_fp(got.cpu().numpy(), ref[name], name)
 
-    # oracle chain
-    Wg, Wu, Wd = (onf4.dequantize(*onf4.quantize(c["W"]), *c["W"].shape) for c in (cg, cu, cd))
-    Xh, dYh = _f64(cg["X"]), _f64(cd["dY"])
-    (Ag, Bg), (Au, Bu), (Ad, Bd) = ((_f64(c["A"]), _f64(c["B"])) for c in (cg, cu, cd))
-    go = _bf16r(olin.linear_fwd(Wg, Xh, Ag, Bg, s)[0])
-    uo = _bf16r(olin.linear_fwd(Wu, Xh, Au, Bu, s)[0])
-    silu = go / (1.0 + np.exp(-go))
-    ho = _bf16r(silu * uo)
-    yo = olin.linear_fwd(Wd, ho, Ad, Bd, s)[0]
-    dho, dAdo, dBdo = olin.linear_bwd(Wd, ho, Ad, Bd, s, dYh)
-    dho = _bf16r(dho)
-    sg = 1.0 / (1.0 + np.exp(-go))
-    dgo = _bf16r(dho * uo * sg * (1 + go * (1 - sg)))
-    duo = _bf16r(dho * silu)
-    dXgo, dAgo, dBgo = olin.linear_bwd(Wg, Xh, Ag, Bg, s, dgo)
-    dXuo, dAuo, dBuo = olin.linear_bwd(Wu, Xh, Au, Bu, s, duo)
 
-    assert_close_fp(bf16_dev_to_f64(g), go, "gate output")
-    assert_close_fp(bf16_dev_to_f64(h), ho, "SiLU(g) * u")
-    assert_close_fp(bf16_dev_to_f64(y), yo, "MLP output")
-    assert_close_fp(bf16_dev_to_f64(dh), dho, "dH")
-    assert_close_fp(dX.double().cpu().numpy(), dXgo + dXuo, "dX")
-    for name, got, ref in (("dA down", dAd, dAdo), ("dB down", dBd, dBdo), ("dA gate", dAg, dAgo),
-                           ("dB gate", dBg, dBgo), ("dA up", dAu, dAuo), ("dB up", dBu, dBuo)):
-        assert_close_fp(got.cpu().numpy(), ref, name)
+def test_mlp_7b_chain_fused_swiglu(lib, mlp_7b):
+    """The same chain with gate and up fused: one GEMM over the interleaved
+    NF4 weight writes h = silu(g) * u, the recompute repeats it (same bits),
+    and the backward's fused GEMM recomputes g and u to write dg and du; dX
+    and the adapter gradients follow from the existing kernels over the fused
+    operands. Checked against the same oracle chain."""
+    import torch
+    d, s, r = mlp_7b, mlp_7b["s"], mlp_7b["r"]
+    cg, cu, cd = d["cg"], d["cu"], d["cd"]
+    X = to_dev_bf16(d["X"])
+    dY = to_dev_bf16(d["dY"])
+    M, K = X.shape
+    Fd = cg["W"].shape[0]
+    qgu = lib.nf4_quantize(lib.swiglu_interleave(torch.from_numpy(cg["W"]), torch.from_numpy(cu["W"])).cuda())
+    qd = lib.nf4_quantize(torch.from_numpy(cd["W"]).cuda())
+    Agu = to_dev_bf16(np.concatenate([cg["A"], cu["A"]]))
+    Bgu = lib.swiglu_pack_b(to_dev_bf16(cg["B"]), to_dev_bf16(cu["B"]))
+    Ad, Bd = to_dev_bf16(cd["A"]), to_dev_bf16(cd["B"])
+    ws = torch.empty(lib.linear_workspace(M, 2 * Fd, K, 2 * r), dtype=torch.uint8, device="cuda")
+    sUgu = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
+    lib.lora_xa(X, Agu, s, sUgu, ws)
+    h = lib.swiglu_fwd(qgu, X, Bgu, sUgu)
+    y, sUd = lib.linear_fwd(qd, h, Ad, Bd, s)
+    h2 = lib.swiglu_fwd(qgu, X, Bgu, sUgu)        # recompute before the backward
+    torch.cuda.synchronize()
+    assert torch.equal(h, h2)
+    dh, dAd, dBd = lib.linear_bwd(qd, h2, Ad, Bd, s, dY, sU=sUd)
+    dGU = lib.swiglu_bwd(qgu, X, Bgu, sUgu, dh)
+    sTgu = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
+    lib.lora_dyb(dGU, Bgu, s, sTgu, ws)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    lib.fused_dx(qgu, dGU, Agu, sTgu, dX)
+    dAgu = torch.empty((2 * r, K), dtype=torch.float32, device="cuda")
+    dBgu = torch.empty((2 * Fd, 2 * r), dtype=torch.float32, device="cuda")
+    lib.lora_grads(X, dGU, sUgu, sTgu, dAgu, dBgu, ws)
+    dBg, dBu = lib.swiglu_unpack_db(dBgu)
+    torch.cuda.synchronize()
+    ref = d["ref"]
+    assert_close_fp(bf16_dev_to_f64(h), ref["h"], "SiLU(g) * u (fused)")
+    assert_close_fp(bf16_dev_to_f64(y), ref["y"], "MLP output")
+    assert_close_fp(bf16_dev_to_f64(dh), ref["dh"], "dH")
+    assert_close_fp(bf16_dev_to_f64(dX), ref["dX"], "dX (fused)")
+    dA = dAgu.cpu().numpy()
+    for name, got in (("dAd", dAd.cpu().numpy()), ("dBd", dBd.cpu().numpy()), ("dAg", dA[:r]), ("dAu", dA[r:]),
+                      ("dBg", dBg.cpu().numpy()), ("dBu", dBu.cpu().numpy())):
+        assert_close_fp(got, ref[name], name + " (fused)")
