@@ -297,6 +297,40 @@ def bench_dequant(q, torch, mats, steps, warmup):
             "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats)}
 
 
+def bench_merge(q, torch, mats, steps, warmup):
+    """Adapter merge W' + s B A to bf16 over the 8B set (r=16): HBM-bound like
+    the standalone dequantisation (0.516 B read + 2 B written per weight)."""
+    r, s = 16, 2.0
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    outs = [torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device="cuda") for lin, _ in mats]
+    adapters = {}
+    for lin, _ in mats:
+        if (lin.N, lin.K) not in adapters:
+            adapters[(lin.N, lin.K)] = ((torch.randn((r, lin.K), generator=g, device="cuda") / r).bfloat16(),
+                                        (torch.randn((lin.N, r), generator=g, device="cuda") * 0.01).bfloat16())
+    moved = sum(lin.N * lin.K * 2 + sum(q.nf4_sizes(lin.N, lin.K)) + 2 * r * (lin.N + lin.K) for lin, _ in mats)
+
+    def one_pass():
+        for (lin, m), o in zip(mats, outs):
+            A, B = adapters[(lin.N, lin.K)]
+            q.nf4_merge(m, A, B, s, out=o)
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one_pass()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del outs
+    return {"workload": "set_8b merge W' + s B A (r=16) of 224 matrices to bf16", "GB/s": moved / ms / 1e6,
+            "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats)}
+
+
 def bench_decode(q, torch, mats, steps, warmup):
     from bit_nf4_quantized_dequant_b200 import inputs
     M, r = 8, 16
@@ -619,6 +653,9 @@ def main():
         mats = eight_b_set(q, torch)
         extras["dequant"] = bench_dequant(q, torch, mats, steps=5, warmup=2)
         extras["dequant"]["frac_of_hbm"] = extras["dequant"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
+        torch.cuda.empty_cache()
+        extras["merge"] = bench_merge(q, torch, mats, steps=5, warmup=2)
+        extras["merge"]["frac_of_hbm"] = extras["merge"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
         extras["decode_fwd"] = bench_decode(q, torch, mats, steps=5, warmup=2)
         extras["decode_fwd"]["frac_of_hbm"] = extras["decode_fwd"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
         del mats

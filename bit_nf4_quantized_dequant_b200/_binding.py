@@ -19,6 +19,7 @@ __all__ = [
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
     "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
+    "nf4_merge",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +38,7 @@ SYMBOLS = [
     "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
     "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
     "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
+    "qlora_nf4_merge",
 ]
 
 
@@ -101,6 +103,9 @@ def library():
     lib.qlora_swiglu_pack_b.restype = st
     lib.qlora_swiglu_unpack_db.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
     lib.qlora_swiglu_unpack_db.restype = st
+    lib.qlora_nf4_merge.argtypes = [ctypes.POINTER(_NF4), _P, _P, ctypes.c_int32, ctypes.c_float, _P, ctypes.c_int32,
+                                    _P]
+    lib.qlora_nf4_merge.restype = st
     lib.qlora_fused_workspace.argtypes = [_I64, ctypes.POINTER(_SZ)]
     lib.qlora_fused_workspace.restype = st
     lib.qlora_fused_fwd.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, ctypes.c_int32, _P, _P, _P, _SZ, _P, _P]
@@ -372,3 +377,14 @@ def swiglu_bwd(q: NF4Matrix, X, Bgu, sUgu, dH, dGU=None, status=None, stream=Non
     _check(library().qlora_swiglu_bwd(ctypes.byref(st), _ptr(X), M, _ptr(Bgu), Bgu.shape[1], _ptr(sUgu), _ptr(dH),
                                       _ptr(dGU), _ptr(status), _stream(stream)), "qlora_swiglu_bwd")
     return dGU
+
+
+def nf4_merge(q: NF4Matrix, A, B, s: float, out=None, f32: bool = False, stream=None):
+    """W' + s B A as bf16 (or fp32 with f32=True) [rows, cols]."""
+    import torch
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.float32 if f32 else torch.bfloat16, device=A.device)
+    st = q.c_struct()
+    _check(library().qlora_nf4_merge(ctypes.byref(st), _ptr(A), _ptr(B), A.shape[0], s, _ptr(out), 1 if f32 else 0,
+                                     _stream(stream)), "qlora_nf4_merge")
+    return out

@@ -374,6 +374,17 @@ qlora_status_t qlora_swiglu_unpack_db(const float *dBgu, int64_t F, int32_t r, f
   return cuda_status(launch_swiglu_unpack_db(dBgu, F, r, dBg, dBu, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_nf4_merge(const qlora_nf4_t *W, const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                               void *out, int32_t out_f32, qlora_stream_t stream) {
+  qlora_status_t st = check_nf4(W);
+  if (st != QLORA_OK) return st;
+  if (!A || !B || !out || !std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  if (W->rows % 16 || r < 1 || r > 64) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_nf4_merge(W->codes, W->scale8, W->scale2, W->rows, W->cols, A, B, r, s, out,
+                                      out_f32 != 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *qlora_status_string(qlora_status_t status) {
   switch (status) {
     case QLORA_OK: return "QLORA_OK";

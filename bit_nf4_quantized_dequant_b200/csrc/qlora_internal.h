@@ -56,6 +56,11 @@ cudaError_t launch_nf4_gemv_fwd(const uint8_t *codes, const uint8_t *scale8, con
 #include "qlora.h"
 
 namespace qlora {
+// W' + s B A (bf16 or fp32 out), see nf4_merge.cu.
+cudaError_t launch_nf4_merge(const uint8_t *codes, const uint8_t *scale8, const float *scale2, int64_t N, int64_t K,
+                             const uint16_t *Al, const uint16_t *Bl, int r, float s, void *out, bool f32_out,
+                             cudaStream_t st);
+
 // SwiGLU layout helpers (see swiglu_pack.cu).
 cudaError_t launch_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t F, int r, uint16_t *Bgu,
                                  cudaStream_t st);

@@ -250,6 +250,18 @@ qlora_status_t qlora_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64
 qlora_status_t qlora_swiglu_unpack_db(const float *dBgu, int64_t F, int32_t r, float *dBg, float *dBu,
                                       qlora_stream_t stream);
 
+/* Merge the adapter into the base: out = W' + s B A with W' the dequantised
+ * NF4 weight [N, K], A [r, K] and B [N, r] device bf16 ("QLoRA"
+ * (guide.dupenodi.dev), section "Walking through the tooling": merge
+ * W' = W + scaled BA for serving; "QLoRA, in depth", section "Shipping:
+ * merge, re-quantize, verify"). Per element fp32(w') + s * sum_j B A (fp32
+ * accumulation), written as bf16 (round to nearest even) when out_f32 == 0 or
+ * as fp32 otherwise (the input of a re-quantisation with qlora_nf4_quantize).
+ * N % 16 == 0, 1 <= r <= 64, out 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+qlora_status_t qlora_nf4_merge(const qlora_nf4_t *W, const uint16_t *A, const uint16_t *B, int32_t r, float s,
+                               void *out, int32_t out_f32, qlora_stream_t stream);
+
 /*
  * Allocation-free forward. The pages have no counterpart to this call: it is an
  * interface convenience of this library for callers that cannot allocate
