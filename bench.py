@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-extras", action="store_true", help="skip the 8B-set dequant / decode lines")
@@ -393,6 +393,19 @@ def bench_decode(q, torch, mats, steps, warmup):
                          "peak_kind": "64 lanes/clk/SM x SMs x 1965 MHz (max SM clock)"}}
 
 
+def codec_error(q, torch):
+    """RMSE of NF4 and of the evenly spaced int4 comparison codebook (same
+    format) on the attention-projection weight, through the GPU codecs."""
+    from bit_nf4_quantized_dequant_b200 import inputs
+    W = torch.from_numpy(inputs.weight_f32(4096, 4096, index=0, outliers=True)).cuda()
+    out = {"workload": "attn_proj_7b weight 4096x4096, N(0, 0.02) with 0.1% x8 outliers"}
+    for name, book in (("nf4", q.CODEBOOK_NF4), ("int4", q.CODEBOOK_INT4)):
+        back = q.codec_dequantize(q.codec_quantize(W, book), book).float()
+        out[f"rmse_{name}"] = torch.sqrt(torch.mean((back - W) ** 2)).item()
+    out["nf4_over_int4"] = out["rmse_nf4"] / out["rmse_int4"]
+    return out
+
+
 def bench_mlp_chain(q, torch, steps, warmup):
     """Llama-7B SiLU-gated MLP (gate/up 4096->11008, down 11008->4096), 4096
     tokens, r=16, alpha=32, one training step with gradient checkpointing:
@@ -661,6 +674,7 @@ def main():
         del mats
         torch.cuda.empty_cache()
         extras["mlp_chain"] = bench_mlp_chain(q, torch, steps=5, warmup=2)
+        extras["codec_error"] = codec_error(q, torch)
     sampler.close()
 
     cpu = None

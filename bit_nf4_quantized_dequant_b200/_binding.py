@@ -19,7 +19,7 @@ __all__ = [
     "linear_workspace", "linear_fwd", "linear_bwd", "status_string", "STATUS",
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
     "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
-    "nf4_merge",
+    "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +38,7 @@ SYMBOLS = [
     "qlora_lora_xa", "qlora_fused_fwd", "qlora_lora_dyb", "qlora_fused_dx", "qlora_lora_grads",
     "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
     "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
-    "qlora_nf4_merge",
+    "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
 ]
 
 
@@ -103,6 +103,12 @@ def library():
     lib.qlora_swiglu_pack_b.restype = st
     lib.qlora_swiglu_unpack_db.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
     lib.qlora_swiglu_unpack_db.restype = st
+    lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
+    lib.qlora_codec_levels.restype = st
+    lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
+    lib.qlora_codec_quantize.restype = st
+    lib.qlora_codec_dequantize.argtypes = [ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
+    lib.qlora_codec_dequantize.restype = st
     lib.qlora_nf4_merge.argtypes = [ctypes.POINTER(_NF4), _P, _P, ctypes.c_int32, ctypes.c_float, _P, ctypes.c_int32,
                                     _P]
     lib.qlora_nf4_merge.restype = st
@@ -387,4 +393,33 @@ def nf4_merge(q: NF4Matrix, A, B, s: float, out=None, f32: bool = False, stream=
     st = q.c_struct()
     _check(library().qlora_nf4_merge(ctypes.byref(st), _ptr(A), _ptr(B), A.shape[0], s, _ptr(out), 1 if f32 else 0,
                                      _stream(stream)), "qlora_nf4_merge")
+    return out
+
+
+CODEBOOK_NF4, CODEBOOK_INT4 = 0, 1
+
+
+def codec_levels(codebook: int):
+    out = (ctypes.c_float * 16)()
+    _check(library().qlora_codec_levels(codebook, out), "qlora_codec_levels")
+    return list(out)
+
+
+def codec_quantize(W, codebook: int, out: NF4Matrix | None = None, status=None, stream=None) -> NF4Matrix:
+    """Quantise with NF4 or the evenly spaced int4 comparison codebook (same format)."""
+    rows, cols = W.shape
+    q = out if out is not None else NF4Matrix.empty(rows, cols, W.device)
+    s = q.c_struct()
+    _check(library().qlora_codec_quantize(_ptr(W), ctypes.byref(s), codebook, _ptr(status), _stream(stream)),
+           "qlora_codec_quantize")
+    return q
+
+
+def codec_dequantize(q: NF4Matrix, codebook: int, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.codes.device)
+    s = q.c_struct()
+    _check(library().qlora_codec_dequantize(ctypes.byref(s), codebook, _ptr(out), _stream(stream)),
+           "qlora_codec_dequantize")
     return out

@@ -166,6 +166,38 @@ qlora_status_t qlora_nf4_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora_s
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_codec_levels(int32_t codebook, float *out) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  static const float nf4[16] = QLORA_NF4_LEVELS;
+  static const float int4[16] = QLORA_INT4_LEVELS;
+  if (codebook == QLORA_CODEBOOK_NF4) std::memcpy(out, nf4, sizeof(nf4));
+  else if (codebook == QLORA_CODEBOOK_INT4) std::memcpy(out, int4, sizeof(int4));
+  else return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_codec_quantize(const float *W, const qlora_nf4_t *q, int32_t codebook, int32_t *dev_status,
+                                    qlora_stream_t stream) {
+  if (codebook != QLORA_CODEBOOK_NF4 && codebook != QLORA_CODEBOOK_INT4) return QLORA_ERR_INVALID_ARG;
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_quantize(W, q->rows, q->cols, q->codes, q->scale8, q->scale2, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream), codebook));
+}
+
+qlora_status_t qlora_codec_dequantize(const qlora_nf4_t *q, int32_t codebook, uint16_t *out, qlora_stream_t stream) {
+  if (codebook != QLORA_CODEBOOK_NF4 && codebook != QLORA_CODEBOOK_INT4) return QLORA_ERR_INVALID_ARG;
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(out)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_dequantize(q->codes, q->scale8, q->scale2, q->rows, q->cols, out,
+                                       reinterpret_cast<cudaStream_t>(stream), codebook));
+}
+
 qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t *bytes) {
   if (!bytes || M <= 0 || N <= 0 || K <= 0) return QLORA_ERR_INVALID_ARG;
   if (K % kBlock || N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;

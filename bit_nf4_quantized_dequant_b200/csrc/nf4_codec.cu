@@ -13,8 +13,11 @@ namespace {
 // code = number of midpoints between adjacent levels that n lies strictly
 // above: the nearest level, ties to the lower one. The midpoints of two float32
 // levels are exact in float64, and so is the comparison.
+template <int BOOK>
 __device__ __forceinline__ uint32_t nearest_level(float n) {
-  constexpr float L[16] = QLORA_NF4_LEVELS;
+  constexpr float NF4[16] = QLORA_NF4_LEVELS;
+  constexpr float INT4[16] = QLORA_INT4_LEVELS;
+  const float *L = BOOK == kBookInt4 ? INT4 : NF4;
   const double x = static_cast<double>(n);
   uint32_t code = 0;
 #pragma unroll
@@ -28,6 +31,7 @@ __device__ __forceinline__ uint32_t nearest_level(float n) {
 // One CTA per group of 256 blocks; warp w handles blocks w, w+8, ...; lane l
 // holds elements 2l and 2l+1 of a block, so the packed byte l of the block is
 // written by lane l.
+template <int BOOK>
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restrict__ W, int64_t nb,
                                                            uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scale8,
@@ -49,10 +53,11 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
     float m = fmaxf(fabsf(v.x), fabsf(v.y));
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    uint32_t e0 = 7, e1 = 7;
+    constexpr uint32_t kZero = BOOK == kBookInt4 ? 8u : 7u;   // index of the exact zero level
+    uint32_t e0 = kZero, e1 = kZero;
     if (m > 0.f) {
-      e0 = nearest_level(__fdiv_rn(v.x, m));
-      e1 = nearest_level(__fdiv_rn(v.y, m));
+      e0 = nearest_level<BOOK>(__fdiv_rn(v.x, m));
+      e1 = nearest_level<BOOK>(__fdiv_rn(v.y, m));
     }
     codes[b * (kBlock / 2) + lane] = static_cast<uint8_t>((e0 << 4) | e1);
     if (lane == 0) c1s[i] = m;
@@ -88,6 +93,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
 // Each warp stages its 32 x 64 contiguous output bytes in shared memory and
 // writes them with one bulk copy, so global stores are full, contiguous 2 KiB
 // runs instead of 64-byte pieces strided across the warp.
+template <int BOOK>
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
                                                           const uint8_t *__restrict__ scale8,
                                                           const float *__restrict__ scale2,
@@ -103,7 +109,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
     const int64_t b = i >> 1;
     const uint4 c = __ldg(reinterpret_cast<const uint4 *>(codes) + i);
     const float sc = block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
-    const Nf4Table t = make_table(sc);
+    const Nf4Table t = make_table_book<BOOK>(sc);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -125,23 +131,28 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
-                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s) {
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book) {
   const int64_t nb = rows * cols / kBlock;
   const int64_t ng = (nb + kGroup - 1) / kGroup;
   if (dev_status) {
     cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
   }
-  nf4_quantize_kernel<<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2,
-                                                                dev_status);
+  if (book == kBookInt4)
+    nf4_quantize_kernel<kBookInt4><<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+  else
+    nf4_quantize_kernel<kBookNf4><<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
-                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s) {
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book) {
   const int64_t nhalf = rows * cols / 32;
   const int64_t grid = (nhalf + 255) / 256;
-  nf4_dequant_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+  if (book == kBookInt4)
+    nf4_dequant_kernel<kBookInt4><<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+  else
+    nf4_dequant_kernel<kBookNf4><<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
   return cudaGetLastError();
 }
 

@@ -24,6 +24,21 @@ namespace qlora {
    0x1.45f602p-4f,  0x1.4995bep-3f,  0x1.f809b4p-3f,  0x1.5a066cp-2f,        \
    0x1.c3496ap-2f,  0x1.200f52p-1f,  0x1.722760p-1f,  0x1.000000p+0f}
 
+// Comparison codebook: evenly spaced int4 levels (k - 8) / 7, k = 0..15, as
+// float32 ("What is QLoRA ...", "Follow-up questions to expect": plain int4
+// spaces its levels evenly and wastes them on rare large values). The same
+// block constants and 8-bit double quantisation apply; code 8 is zero and
+// level 0 (-8/7) is never chosen, since |w / c1| <= 1.
+#define QLORA_INT4_LEVELS                                                    \
+  {-0x1.24924ap+0f, -0x1.000000p+0f, -0x1.b6db6ep-1f, -0x1.6db6dcp-1f,       \
+   -0x1.24924ap-1f, -0x1.b6db6ep-2f, -0x1.24924ap-2f, -0x1.24924ap-3f,       \
+   0x0.0p+0f,       0x1.24924ap-3f,  0x1.24924ap-2f,  0x1.b6db6ep-2f,        \
+   0x1.24924ap-1f,  0x1.6db6dcp-1f,  0x1.b6db6ep-1f,  0x1.000000p+0f}
+
+// Codebook identifiers (the values of qlora_codebook_t).
+constexpr int kBookNf4 = 0;
+constexpr int kBookInt4 = 1;
+
 // ---------------------------------------------------------------------------
 // Small PTX wrappers
 // ---------------------------------------------------------------------------
@@ -439,8 +454,7 @@ __device__ __forceinline__ float block_scale(uint32_t q8, float d) {
   return __fmul_rn(static_cast<float>(q8), d);
 }
 
-__device__ __forceinline__ Nf4Table make_table(float s) {
-  constexpr float L[16] = QLORA_NF4_LEVELS;
+__device__ __forceinline__ Nf4Table table_from_levels(const float (&L)[16], float s) {
   uint32_t pk[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__fmul_rn(L[2 * i], s), __fmul_rn(L[2 * i + 1], s));
@@ -453,6 +467,19 @@ __device__ __forceinline__ Nf4Table make_table(float s) {
   }
   return t;
 }
+
+template <int BOOK>
+__device__ __forceinline__ Nf4Table make_table_book(float s) {
+  if constexpr (BOOK == kBookInt4) {
+    constexpr float L[16] = QLORA_INT4_LEVELS;
+    return table_from_levels(L, s);
+  } else {
+    constexpr float L[16] = QLORA_NF4_LEVELS;
+    return table_from_levels(L, s);
+  }
+}
+
+__device__ __forceinline__ Nf4Table make_table(float s) { return make_table_book<kBookNf4>(s); }
 
 // Expand one 32-bit word of packed codes (8 weights, element 2j in the high
 // nibble of byte j) into 8 bf16 values, returned as 4 words of bf16 pairs in

@@ -11,10 +11,11 @@ constexpr int kBlock = 64;    // weights per first-level block
 constexpr int kGroup = 256;   // blocks per second-level group
 
 // Kernel launchers. Each returns the cudaError_t of the launch.
+// book: 0 = NF4, 1 = the evenly spaced int4 comparison codebook.
 cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
-                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s);
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book = 0);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
-                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s);
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book = 0);
 
 // Fused NF4 GEMM (tcgen05). Mode FWD: Y[M,N] = X[M,K] W'^T + sU[M,r] Bl^T.
 // Mode DX: dX[M,K] = dY[M,N] W' + sT[M,r] Al.

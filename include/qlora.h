@@ -102,6 +102,25 @@ qlora_status_t qlora_nf4_quantize(const float *W, const qlora_nf4_t *q,
 qlora_status_t qlora_nf4_dequantize(const qlora_nf4_t *q, uint16_t *out,
                                     qlora_stream_t stream);
 
+/* Comparison codec. The same stored format (packed 4-bit codes, 8-bit block
+ * constants, fp32 second-level scales) with another 16-level codebook, so
+ * that the error NF4 saves can be measured ("What is QLoRA ...",
+ * "Follow-up questions to expect": evenly spaced int4 levels waste levels on
+ * rare large values, NF4 follows the bell-shaped weights and errs less).
+ * QLORA_CODEBOOK_NF4 is the codebook of qlora_nf4_quantize/dequantize;
+ * QLORA_CODEBOOK_INT4 has the levels (k - 8) / 7, k = 0..15 (fp32), zero at
+ * code 8. Encoding rules, ties and the double quantisation are those of NF4. */
+typedef enum { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_INT4 = 1 } qlora_codebook_t;
+
+/* The 16 fp32 levels of a codebook (host). Errors: INVALID_ARG. */
+qlora_status_t qlora_codec_levels(int32_t codebook, float *out);
+
+/* As qlora_nf4_quantize / qlora_nf4_dequantize with the given codebook.
+ * Errors: as those calls, and INVALID_ARG for an unknown codebook. */
+qlora_status_t qlora_codec_quantize(const float *W, const qlora_nf4_t *q, int32_t codebook, int32_t *dev_status,
+                                    qlora_stream_t stream);
+qlora_status_t qlora_codec_dequantize(const qlora_nf4_t *q, int32_t codebook, uint16_t *out, qlora_stream_t stream);
+
 /* Workspace bytes that qlora_linear_fwd and qlora_linear_bwd need for M
  * tokens through an [N, K] layer of rank r (host). The same workspace may be
  * reused by consecutive calls on one stream; calls that run concurrently need
