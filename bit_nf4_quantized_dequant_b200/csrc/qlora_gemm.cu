@@ -184,7 +184,9 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int slots, uint32_t i
   }
 }
 
-template <bool kPair>
+// One instantiation per (pair, mode, stream-K) so that each launch carries only
+// the code of its own epilogue: the instruction cache is shared by all roles.
+template <bool kPair, int kMode, bool kStreamK>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                           const __grid_constant__ CUtensorMap tm_codes,
@@ -198,8 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Smem sm = carve(base, p);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool dx = p.mode == 1;
-  const bool swiglu = p.mode >= 2;
+  constexpr bool dx = kMode == 1;
+  constexpr bool swiglu = kMode >= 2;
   // CTA pair: rank 0 (even CTA) issues the MMAs; rank 1 is its peer.
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t units = static_cast<int64_t>(ntiles) * p.nk;
   // first unit of CTA j under the stream-K split
   auto unit_begin = [&](int64_t j) -> int64_t { return units * j / gridDim.x; };
-  if (!kPair && p.streamk) {
+  if constexpr (!kPair && kStreamK) {
     const int64_t u0 = unit_begin(blockIdx.x), u1 = unit_begin(blockIdx.x + 1);
     walk.first_tile = static_cast<int>(u0 / p.nk);
     walk.first_k = static_cast<int>(u0 % p.nk);
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_lora_w);
     tma_prefetch_desc(&tm_lora_act);
     tma_prefetch_desc(&tm_out);
-    if (p.mode == 3) tma_prefetch_desc(&tm_aux);
+    if constexpr (kMode == 3) tma_prefetch_desc(&tm_aux);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -454,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kb = seg.k;
       const int len = p.nk - kb < total_steps - done ? p.nk - kb : total_steps - done;
       const int rt = seg.rt, tt = seg.tt;
-      const bool head = kb > 0;                  // the end of a tile whose start another CTA computes
-      const bool tail = kb + len < p.nk;         // the start of a tile that the next CTA completes
+      const bool head = kStreamK && kb > 0;             // the end of a tile whose start another CTA computes
+      const bool tail = kStreamK && kb + len < p.nk;    // the start of a tile that the next CTA completes
       const int buf = si & 1;
       if (!mbar_wait(&sm.accf[buf], static_cast<uint32_t>(si >> 1) & 1u, abort_flag, p.status)) break;
       tc_fence_after();
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto dh_buf = [&](uint32_t k) {
           return reinterpret_cast<uint16_t *>(sm.out + kOutStageBytes + (k & 1u) * (kOutStageBytes / 2));
         };
-        if (p.mode == 3 && et == 0) {   // dH for the first 32 tokens of the tile
+        if (kMode == 3 && et == 0) {   // dH for the first 32 tokens of the tile
           mbar_arrive_expect_tx(&sm.dhf[dh_count & 1u], dh_bytes);
           tma_load_2d(dh_buf(dh_count), &tm_aux, &sm.dhf[dh_count & 1u], rt * 64, tt * p.bt);
         }
@@ -524,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) arrive_leader(&sm.acce[buf]);
           }
-          if (p.mode == 2) {
+          if constexpr (kMode == 2) {
             // h = bf16(silu(g) * u) -> H[tokens, 64 columns]
             uint8_t *cb = sm.out + (chunk_count & 1u) * kOutStageBytes;
             uint16_t *ux = reinterpret_cast<uint16_t *>(cb);          // [32 tokens][64] u
@@ -901,9 +903,6 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   const int ntiles = p.row_tiles * p.tok_tiles;
   const int sms = device_sm_count();
   if (!pair) {
-    cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
     int grid = ntiles < sms ? ntiles : sms;
     if (a.ws && bt <= 64 && a.mode <= 1) {
       // Stream-K over all SMs for short token tiles: a few weight-row tiles
@@ -919,10 +918,26 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
       p.flags = static_cast<uint64_t *>(a.ws);
       p.part = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + flags);
     }
-    fused_nf4_gemm_kernel<false><<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux, p);
-    return cudaGetLastError();
+    auto go = [&](auto kernel) -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      kernel<<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux, p);
+      return cudaGetLastError();
+    };
+    switch (a.mode * 2 + p.streamk) {
+      case 0: return go(fused_nf4_gemm_kernel<false, 0, false>);
+      case 1: return go(fused_nf4_gemm_kernel<false, 0, true>);
+      case 2: return go(fused_nf4_gemm_kernel<false, 1, false>);
+      case 3: return go(fused_nf4_gemm_kernel<false, 1, true>);
+      case 4: return go(fused_nf4_gemm_kernel<false, 2, false>);
+      case 6: return go(fused_nf4_gemm_kernel<false, 3, false>);
+      default: return cudaErrorInvalidValue;
+    }
   }
-  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (a.mode > 1) return cudaErrorInvalidValue;
+  const void *pair_fn = a.mode == 0 ? reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true, 0, false>)
+                                    : reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true, 1, false>);
+  cudaError_t e = cudaFuncSetAttribute(pair_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int pairs = ntiles < sms / 2 ? ntiles : sms / 2;
@@ -939,7 +954,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void *args[] = {&tm_act, &tm_codes, &tm_lw, &tm_la, &tm_out, &tm_aux, &p};
-  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true>), args);
+  return cudaLaunchKernelExC(&cfg, pair_fn, args);
 }
 
 }  // namespace qlora
