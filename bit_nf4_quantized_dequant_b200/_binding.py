@@ -20,6 +20,7 @@ __all__ = [
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
     "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
+    "adamw8_step", "AdamW8State",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +40,7 @@ SYMBOLS = [
     "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
     "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
     "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
+    "qlora_adamw8_step",
 ]
 
 
@@ -103,6 +105,9 @@ def library():
     lib.qlora_swiglu_pack_b.restype = st
     lib.qlora_swiglu_unpack_db.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
     lib.qlora_swiglu_unpack_db.restype = st
+    lib.qlora_adamw8_step.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, ctypes.c_int32, ctypes.c_float,
+                                      ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P]
+    lib.qlora_adamw8_step.restype = st
     lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_codec_levels.restype = st
     lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
@@ -423,3 +428,26 @@ def codec_dequantize(q: NF4Matrix, codebook: int, out=None, stream=None):
     _check(library().qlora_codec_dequantize(ctypes.byref(s), codebook, _ptr(out), _stream(stream)),
            "qlora_codec_dequantize")
     return out
+
+
+class AdamW8State:
+    """8-bit AdamW states of one parameter tensor (zero-initialised)."""
+
+    def __init__(self, numel: int, device="cuda"):
+        import torch
+        blocks = -(-numel // 256)
+        self.m_q = torch.zeros(numel, dtype=torch.int8, device=device)
+        self.v_q = torch.zeros(numel, dtype=torch.uint8, device=device)
+        self.m_scale = torch.zeros(blocks, dtype=torch.float32, device=device)
+        self.v_scale = torch.zeros(blocks, dtype=torch.float32, device=device)
+        self.step = 0
+
+
+def adamw8_step(p, grad, state: AdamW8State, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                eps: float = 1e-8, weight_decay: float = 0.0, p_bf16=None, stream=None):
+    """One AdamW step on fp32 p (in place) with 8-bit states; optional bf16 copy."""
+    state.step += 1
+    _check(library().qlora_adamw8_step(_ptr(p), _ptr(p_bf16), _ptr(grad), _ptr(state.m_q), _ptr(state.v_q),
+                                       _ptr(state.m_scale), _ptr(state.v_scale), p.numel(), state.step, lr, beta1,
+                                       beta2, eps, weight_decay, _stream(stream)), "qlora_adamw8_step")
+    return p

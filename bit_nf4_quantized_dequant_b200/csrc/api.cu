@@ -417,6 +417,17 @@ qlora_status_t qlora_nf4_merge(const qlora_nf4_t *W, const uint16_t *A, const ui
                                       out_f32 != 0, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_adamw8_step(float *p, uint16_t *p_bf16, const float *grad, int8_t *m_q, uint8_t *v_q,
+                                 float *m_scale, float *v_scale, int64_t n, int32_t step, float lr, float beta1,
+                                 float beta2, float eps, float weight_decay, qlora_stream_t stream) {
+  if (!p || !grad || !m_q || !v_q || !m_scale || !v_scale || n <= 0 || step < 1) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(lr) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps > 0.f) ||
+      !std::isfinite(weight_decay))
+    return QLORA_ERR_INVALID_ARG;
+  return cuda_status(launch_adamw8(p, p_bf16, grad, m_q, v_q, m_scale, v_scale, n, step, lr, beta1, beta2, eps,
+                                   weight_decay, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char *qlora_status_string(qlora_status_t status) {
   switch (status) {
     case QLORA_OK: return "QLORA_OK";

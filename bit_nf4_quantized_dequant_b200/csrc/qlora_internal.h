@@ -62,6 +62,11 @@ cudaError_t launch_nf4_merge(const uint8_t *codes, const uint8_t *scale8, const 
                              const uint16_t *Al, const uint16_t *Bl, int r, float s, void *out, bool f32_out,
                              cudaStream_t st);
 
+// AdamW with 8-bit states (blocks of 256), see adamw8.cu.
+cudaError_t launch_adamw8(float *p, uint16_t *p_bf16, const float *grad, int8_t *mq, uint8_t *vq, float *mscale,
+                          float *vscale, int64_t n, int step, float lr, float beta1, float beta2, float eps, float wd,
+                          cudaStream_t st);
+
 // SwiGLU layout helpers (see swiglu_pack.cu).
 cudaError_t launch_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t F, int r, uint16_t *Bgu,
                                  cudaStream_t st);

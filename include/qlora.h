@@ -281,6 +281,26 @@ qlora_status_t qlora_swiglu_unpack_db(const float *dBgu, int64_t F, int32_t r, f
 qlora_status_t qlora_nf4_merge(const qlora_nf4_t *W, const uint16_t *A, const uint16_t *B, int32_t r, float s,
                                void *out, int32_t out_f32, qlora_stream_t stream);
 
+/* One AdamW step (decoupled weight decay) of an adapter parameter with 8-bit
+ * optimiser states ("QLoRA, in depth", section "A complete run on a 12
+ * GB-class GPU": training uses the paged 8-bit AdamW, which keeps its states in
+ * 8 bits; paging is not part of this library). p [n] fp32 master weights,
+ * updated in place; p_bf16 [n] or NULL receives bf16_rn(p) for the kernels;
+ * grad [n] fp32 (e.g. dA or dB from qlora_lora_grads). States in blocks of 256
+ * elements: m_q int8 with m = m_q / 127 * m_scale[block], v_q uint8 codes of
+ * sqrt(v) with v = (v_q / 255)^2 * v_scale[block] (a nonzero v keeps a code
+ * >= 1); zero-initialised states are the usual start.
+ * Per element, in fp32 with every operation rounded once:
+ *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g g;
+ *   p -= lr (m / (1 - b1^t) / (sqrt(v / (1 - b2^t)) + eps) + wd p),
+ * then per block m_scale = max |m|, v_scale = max v and the codes are
+ * rint(127 m / m_scale) and, for v > 0, clamp(rint(255 sqrt(v / v_scale)),
+ * 1, 255) (half to even). step t >= 1.
+ * Errors: INVALID_ARG, CUDA. */
+qlora_status_t qlora_adamw8_step(float *p, uint16_t *p_bf16, const float *grad, int8_t *m_q, uint8_t *v_q,
+                                 float *m_scale, float *v_scale, int64_t n, int32_t step, float lr, float beta1,
+                                 float beta2, float eps, float weight_decay, qlora_stream_t stream);
+
 /*
  * Allocation-free forward. The pages have no counterpart to this call: it is an
  * interface convenience of this library for callers that cannot allocate
