@@ -484,6 +484,61 @@ def bench_mlp_chain(q, torch, steps, warmup):
     return out
 
 
+def bench_stack(q, torch, name, mats, steps, warmup):
+    """fwd+bwd of every linear of a model's linear set (the 3B decoder stack
+    at 2048 tokens, the 8B set at 4096 tokens): each linear is one run_step
+    (the five-launch DAG) over its own NF4 weight and adapter, in layer order.
+    Activations and output gradients rotate over two layers' worth of buffers
+    (several hundred MB, > L2); q, k, v read the same X, as do gate and up."""
+    from bit_nf4_quantized_dequant_b200 import inputs
+    wl = inputs.WORKLOADS[name]
+    M, r, s = wl.M, wl.r, wl.s
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7000)
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, generator=g, device="cuda") * std).bfloat16()
+    if mats is None:
+        mats = []
+        for i, lin in enumerate(wl.linears):
+            Wf = torch.randn((lin.N, lin.K), generator=g, device="cuda", dtype=torch.float32) * 0.02
+            mats.append((lin, q.nf4_quantize(Wf)))
+            del Wf
+    shapes = sorted({(lin.N, lin.K) for lin, _ in mats})
+    acts = [{nk: dict(X=rnd(M, nk[1]), dY=rnd(M, nk[0])) for nk in shapes} for _ in range(2)]
+    e = lambda *shape, dt=torch.bfloat16: torch.empty(*shape, dtype=dt, device="cuda")
+    outs = {(N, K): dict(Y=e(M, N), dX=e(M, K), dA=e(r, K, dt=torch.float32), dB=e(N, r, dt=torch.float32))
+            for N, K in shapes}
+    ws = e(max(q.linear_workspace(M, N, K, r) for N, K in shapes), dt=torch.uint8)
+    gws = e(q.fused_workspace(M), dt=torch.uint8)
+    sU, sT = e(M, r), e(M, r)
+    per_layer = len({lin.name for lin in wl.linears})   # q, k, v, o, gate, up, down
+    steps_d = []
+    for i, (lin, m) in enumerate(mats):
+        nk = (lin.N, lin.K)
+        d = dict(q=m, A=rnd(r, lin.K, std=1 / r), B=rnd(lin.N, r, std=0.01), sU=sU, sT=sT, ws=ws, gws=gws)
+        d.update(acts[(i // per_layer) % 2][nk])
+        d.update(outs[nk])
+        steps_d.append(d)
+    side = make_side(torch)
+
+    def one_pass():
+        for d in steps_d:
+            run_step(q, d, s, side=side)
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one_pass()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    flops = sum(step_flops(M, lin.N, lin.K, r) for lin, _ in mats)
+    return {"workload": wl.description + ", fwd+bwd of every linear (no dW)", "TFLOP/s": flops / (ms * 1e-3) / 1e12,
+            "ms_per_pass": ms, "flops_per_pass": flops, "launches_per_pass": LAUNCHES_PER_STEP * len(mats)}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (bounded sample)
 # ---------------------------------------------------------------------------
@@ -671,7 +726,14 @@ def main():
         extras["merge"]["frac_of_hbm"] = extras["merge"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
         extras["decode_fwd"] = bench_decode(q, torch, mats, steps=5, warmup=2)
         extras["decode_fwd"]["frac_of_hbm"] = extras["decode_fwd"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
+        extras["set_8b_fwd_bwd"] = bench_stack(q, torch, "set_8b", mats, steps=3, warmup=1)
         del mats
+        torch.cuda.empty_cache()
+        extras["stack_3b_fwd_bwd"] = bench_stack(q, torch, "stack_3b", None, steps=3, warmup=1)
+        for k in ("set_8b_fwd_bwd", "stack_3b_fwd_bwd"):
+            extras[k]["frac_of_bf16_burst"] = extras[k]["TFLOP/s"] / peak
+            extras[k]["frac_of_bf16_sustained"] = extras[k]["TFLOP/s"] / peaks.get(
+                "bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         torch.cuda.empty_cache()
         extras["mlp_chain"] = bench_mlp_chain(q, torch, steps=5, warmup=2)
         extras["codec_error"] = codec_error(q, torch)

@@ -20,7 +20,8 @@ __all__ = [
     "lora_xa", "fused_fwd", "lora_dyb", "fused_dx", "lora_grads", "linear_fwd_noalloc",
     "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
-    "adamw8_step", "AdamW8State",
+    "adamw8_step", "AdamW8State", "set_gemm_schedule", "gemm_schedule",
+    "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +41,7 @@ SYMBOLS = [
     "qlora_linear_fwd_noalloc", "qlora_fused_workspace",
     "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
     "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
-    "qlora_adamw8_step",
+    "qlora_adamw8_step", "qlora_set_gemm_schedule",
 ]
 
 
@@ -108,6 +109,8 @@ def library():
     lib.qlora_adamw8_step.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I64, ctypes.c_int32, ctypes.c_float,
                                       ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float, _P]
     lib.qlora_adamw8_step.restype = st
+    lib.qlora_set_gemm_schedule.argtypes = [ctypes.c_int32]
+    lib.qlora_set_gemm_schedule.restype = st
     lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_codec_levels.restype = st
     lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
@@ -451,3 +454,29 @@ def adamw8_step(p, grad, state: AdamW8State, lr: float, beta1: float = 0.9, beta
                                        _ptr(state.m_scale), _ptr(state.v_scale), p.numel(), state.step, lr, beta1,
                                        beta2, eps, weight_decay, _stream(stream)), "qlora_adamw8_step")
     return p
+
+
+# ---------------------------------------------------------------------------
+# fused-GEMM tile schedule (process-wide)
+# ---------------------------------------------------------------------------
+SCHEDULE_AUTO, SCHEDULE_SINGLE, SCHEDULE_PAIR = 0, 1, 2
+
+
+class gemm_schedule:
+    """Context manager that selects the fused GEMM's tile schedule
+    (qlora_set_gemm_schedule) and restores the automatic one on exit."""
+
+    def __init__(self, schedule: int):
+        self.schedule = schedule
+
+    def __enter__(self):
+        set_gemm_schedule(self.schedule)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemm_schedule(SCHEDULE_AUTO)
+        return False
+
+
+def set_gemm_schedule(schedule: int) -> None:
+    _check(library().qlora_set_gemm_schedule(int(schedule)), "qlora_set_gemm_schedule")

@@ -428,6 +428,12 @@ qlora_status_t qlora_adamw8_step(float *p, uint16_t *p_bf16, const float *grad, 
                                    weight_decay, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_set_gemm_schedule(int32_t schedule) {
+  if (schedule < QLORA_SCHEDULE_AUTO || schedule > QLORA_SCHEDULE_PAIR) return QLORA_ERR_INVALID_ARG;
+  qlora::set_gemm_schedule(schedule);
+  return QLORA_OK;
+}
+
 const char *qlora_status_string(qlora_status_t status) {
   switch (status) {
     case QLORA_OK: return "QLORA_OK";

@@ -24,16 +24,23 @@
 // Two groups of four warps dequantise alternate K-steps, one thread per
 // 64-weight block.
 //
-// Two variants share this source. Single CTA: UMMA M = 128, one CTA per tile.
-// CTA pair (cta_group::2, a cluster of two): UMMA M = 256 across the pair; each
-// CTA dequantises its own 128 weight rows and loads half of the token tile.
-// The even CTA issues the MMAs; the odd CTA's producers and dequantisers signal
-// the even CTA's barriers, and the even CTA's MMA completions are multicast to
-// both. The pair halves each SM's activation traffic, but that traffic is not
-// what limits this kernel, and the cluster-scope arrivals cost more than they
-// save, so the launcher dispatches the single-CTA variant.
+// Two variants share this source. Single CTA: UMMA M = 128, one CTA per tile;
+// a K-step of a 256-token tile needs 512 tensor cycles but the dequantisation
+// of its 128 x 64 weights takes longer, so this variant is bound by the
+// dequantisers. CTA pair (cta_group::2, a cluster of two): UMMA M = 256 across
+// the pair and a 512-token tile, issued as two N = 256 MMAs per K-slice into
+// two accumulators that fill each CTA's TMEM; each CTA dequantises its own 128
+// weight rows and loads 256 of the tokens (128 for each MMA), so every
+// dequantised weight feeds twice the flops of the single-CTA tile with the same
+// shared memory per CTA. The even CTA issues the MMAs; the odd CTA's producers
+// and dequantisers signal the even CTA's barriers, and the even CTA's MMA
+// completions are multicast to both; the odd CTA's dequantised tiles reach
+// the even CTA through one forwarding thread (a single cluster-scope release
+// per K-step instead of one per dequantiser warp). On B200 the pair measured
+// no faster than single-CTA tiles (the K-step time grows with its doubled MMA
+// work), so it runs only when the caller selects it (qlora_set_gemm_schedule).
 //
-// Scheduling: persistent CTAs take whole tiles (tile = blockIdx + i * gridDim).
+// Scheduling: persistent CTAs (or pairs) take whole tiles (tile = blockIdx + i * gridDim).
 // With a workspace and token tiles of at most 64, stream-K instead: the
 // (tile, k-step) units are split evenly over all SMs, and tiles cut between
 // CTAs are finished through fp32 partials in the workspace (see GemmParams).
@@ -42,8 +49,10 @@
 // 2 activation producer, 3 LoRA-slice producer, 4-7 epilogue (TMEM lane
 // quadrant = warp % 4; results leave through shared memory and TMA stores),
 // 8-11 and 12-15 the two dequantiser groups. Persistent CTAs walk the tile
-// list; the TMEM accumulator is double-buffered so the epilogue of one tile
-// overlaps the main loop of the next.
+// list; the single-CTA TMEM accumulator is double-buffered so the epilogue of
+// one tile overlaps the main loop of the next (a pair's two accumulators take
+// all 512 columns: its next tile's MMAs wait for the epilogue, while its
+// producers and dequantisers run ahead).
 #include <atomic>
 
 #include "qlora_device.cuh"
@@ -65,8 +74,8 @@ struct GemmParams {
   int32_t *status;
   int64_t N, K, M;
   int mode;        // 0 FWD, 1 DX, 2 SwiGLU FWD (h), 3 SwiGLU BWD (dg, du); 2 and 3 run the FWD main loop
-  int bt;          // token tile of one (pair) tile = UMMA N
-  int bt_cta;      // tokens whose activations this CTA loads (bt, or bt / 2 for a pair)
+  int bt;          // token tile: UMMA N (single CTA), or 512 = two N = 256 MMAs (pair)
+  int bt_cta;      // tokens whose activations this CTA loads (bt, or 256 for a pair)
   int sx, sa, sc;  // ring depths: activations, dequantised tiles, codes
   int r_pad;       // LoRA K extent in smem (16, 32 or 64)
   int row_tiles;   // tiles along the weight dimension (128 rows, or 256 for a pair)
@@ -230,14 +239,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rows_per_tile = kPair ? 2 * kTileRows : kTileRows;
   const int row_off = static_cast<int>(rank) * kTileRows;     // this CTA's weight rows inside the tile
   const int tok_off = static_cast<int>(rank) * p.bt_cta;      // this CTA's tokens inside the tile
-  // two accumulators of bt columns; at least 64 so a 32-column load of buffer 1 stays inside
-  const uint32_t tmem_cols = static_cast<uint32_t>(2 * p.bt) < 64u ? 64u : static_cast<uint32_t>(2 * p.bt);
+  // single CTA: two accumulators of bt columns (at least 64 so a 32-column load
+  // of buffer 1 stays inside); pair: one tile of 512 columns (two N = 256 halves)
+  const uint32_t tmem_cols =
+      kPair ? 512u : (static_cast<uint32_t>(2 * p.bt) < 64u ? 64u : static_cast<uint32_t>(2 * p.bt));
+  // The pair's token order inside a tile: CTA rank q loads tokens [256 q, 256 q + 256)
+  // of the tile; MMA half h reads rows [128 h, 128 h + 128) of both CTAs' stages, so
+  // accumulator column c (half c / 256, n = c % 256) holds token
+  // (n < 128 ? 0 : 256) + 128 (c / 256) + n % 128. A 32-column chunk is 32 consecutive tokens.
+  auto chunk_token = [&](int tt, int col) -> int {
+    if constexpr (kPair) {
+      const int n = col & 255;
+      return tt * p.bt + (n < 128 ? 0 : 256) + 128 * (col >> 8) + (n & 127);
+    } else {
+      return tt * p.bt + col;
+    }
+  };
   volatile int *abort_flag = sm.abort_flag;
 
   if (threadIdx.x == 0) {
-    const uint32_t per_step = kPair ? 8u : 4u;   // dequantiser / epilogue warps that arrive, pair-wide
+    const uint32_t per_step = kPair ? 8u : 4u;   // epilogue warps that arrive, pair-wide
+    // dequantised tile ready: this CTA's four dequantiser warps, plus (even CTA of
+    // a pair) the one forwarded arrival for the odd CTA's half
+    const uint32_t a_arrivals = kPair && leader ? 5u : 4u;
     for (int i = 0; i < p.sx; ++i) { mbar_init(&sm.xf[i], 1); mbar_init(&sm.xe[i], 1); }
-    for (int i = 0; i < p.sa; ++i) { mbar_init(&sm.af[i], per_step); mbar_init(&sm.ae[i], 1); }
+    for (int i = 0; i < p.sa; ++i) { mbar_init(&sm.af[i], a_arrivals); mbar_init(&sm.ae[i], 1); }
     for (int i = 0; i < p.sc; ++i) { mbar_init(&sm.cf[i], 1); mbar_init(&sm.ce[i], 4); }
     mbar_init(sm.lf, 1);
     mbar_init(sm.le, 1);
@@ -362,9 +388,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (the even CTA of a pair) ----------------
+    if (kPair && !leader && elect_one()) {
+      // Odd CTA of a pair: its four dequantiser warps arrive on its own af[slot]
+      // (CTA scope); this thread passes each completed tile on to the even CTA's
+      // af[slot] with one cluster-scope release, which the dequantisers would
+      // otherwise each pay on every K-step.
+      RingPos ar{0, 0};
+      for (int it = 0; it < total_steps; ++it, ar.advance(1, p.sa)) {
+        if (!mbar_wait(&sm.af[ar.slot], ar.phase, abort_flag, p.status)) break;
+        mbar_arrive_cluster(leader_bar(&sm.af[ar.slot]));
+      }
+    }
     if (leader && elect_one()) {
-      const uint32_t idesc =
-          idesc_bf16(static_cast<uint32_t>(rows_per_tile), static_cast<uint32_t>(p.bt), dx, false);
+      const uint32_t idesc = idesc_bf16(static_cast<uint32_t>(rows_per_tile),
+                                        static_cast<uint32_t>(kPair ? 256 : p.bt), dx, false);
       const uint32_t lsw = lora_layout(p.r_pad);
       const uint32_t lsbo = 16u * static_cast<uint32_t>(p.r_pad);   // 8 rows of 2 r_pad bytes
       const uint32_t la_addr = smem_u32(sm.la), lb_addr = smem_u32(sm.lb);
@@ -389,8 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int done = 0, si = 0; done < total_steps && ok; ++si) {
         const int kb = seg.k;
         const int len = p.nk - kb < total_steps - done ? p.nk - kb : total_steps - done;
-        const int buf = si & 1;
-        if (!mbar_wait(&sm.acce[buf], (static_cast<uint32_t>(si >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
+        const int buf = kPair ? 0 : si & 1;
+        const uint32_t acc_ph = kPair ? static_cast<uint32_t>(si) & 1u : static_cast<uint32_t>(si >> 1) & 1u;
+        if (!mbar_wait(&sm.acce[buf], acc_ph ^ 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -410,6 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kKStage / 16; ++j) {
             mma(d_tmem, a0 + static_cast<uint64_t>(a_step * j), b0 + static_cast<uint64_t>(2 * j), (k | j) != 0);
+            if constexpr (kPair)   // tokens of the second half: stage rows 128..255 (+16 KiB)
+              mma(d_tmem + 256u, a0 + static_cast<uint64_t>(a_step * j), b0 + static_cast<uint64_t>(1024 + 2 * j),
+                  (k | j) != 0);
           }
           issued_any = true;
           commit(&sm.xe[xs]);
@@ -425,6 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    : smem_desc(la_addr + 32u * j, 16u, lsbo, lsw);
             const uint64_t bd = smem_desc(lb_addr + 32u * j, 16u, lsbo, lsw);
             mma(d_tmem, ad, bd, 1u);
+            if constexpr (kPair)   // second half: sU / sT rows 128..255
+              mma(d_tmem + 256u, ad, smem_desc(lb_addr + 256u * p.r_pad + 32u * j, 16u, lsbo, lsw), 1u);
           }
           commit(sm.le);
           ++n_lora;
@@ -446,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                 // TMEM lane quadrant of this warp
     const int et = threadIdx.x - 128;       // 0..127 = this CTA's weight row inside the tile
     const int box_t = p.bt < kEpiTokens ? p.bt : kEpiTokens;
-    const int nchunks = p.bt / box_t;
+    const int nchunks = p.bt / box_t;   // a pair's tile: 16 chunks over both halves
     uint32_t chunk_count = 0;
     uint32_t dh_count = 0;   // dH chunk loads so far (SwiGLU backward): buffer and phase
     StepPos seg;
@@ -458,8 +501,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rt = seg.rt, tt = seg.tt;
       const bool head = kStreamK && kb > 0;             // the end of a tile whose start another CTA computes
       const bool tail = kStreamK && kb + len < p.nk;    // the start of a tile that the next CTA completes
-      const int buf = si & 1;
-      if (!mbar_wait(&sm.accf[buf], static_cast<uint32_t>(si >> 1) & 1u, abort_flag, p.status)) break;
+      const int buf = kPair ? 0 : si & 1;
+      const uint32_t acc_ph = kPair ? static_cast<uint32_t>(si) & 1u : static_cast<uint32_t>(si >> 1) & 1u;
+      if (!mbar_wait(&sm.accf[buf], acc_ph, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * p.bt);
@@ -675,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           named_barrier(1, 128);
           if (et == 0) {
-            tma_store_2d(&tm_out, stage, rt * rows_per_tile + row_off, tt * p.bt + c * box_t);
+            tma_store_2d(&tm_out, stage, rt * rows_per_tile + row_off, chunk_token(tt, c * box_t));
             bulk_commit_group();
           }
           __syncwarp();   // reconverge before the next warp-wide TMEM load
@@ -761,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) arrive_leader(&sm.af[as]);
+        if (lane == 0) mbar_arrive(&sm.af[as]);   // CTA scope; the odd CTA's tiles are forwarded
         scale_at(pf, it + 6, qv[u], dv[u]);
         pf.advance(2, p.nk, walk);
         cr.advance(2, p.sc);
@@ -789,6 +833,8 @@ CUtensorMapSwizzle lora_swizzle(int r_pad) {
                      : (r_pad == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+constexpr int kPairRings[3] = {3, 5, 4};   // activation, dequantised-tile, code stages
+
 size_t smem_bytes(int bt_cta, int r_pad, int sx, int sa, int sc) {
   return 1024 /* alignment slack */ + static_cast<size_t>(sx) * bt_cta * 128u +
          static_cast<size_t>(sa) * kATileBytes + lora_b_bytes(bt_cta, r_pad) + lora_a_bytes(r_pad) +
@@ -798,9 +844,17 @@ size_t smem_bytes(int bt_cta, int r_pad, int sx, int sa, int sc) {
 
 // Ring depths that fit the shared-memory budget, in order of preference: at
 // least four activation stages (TMA latency), codes several steps ahead, three
-// dequantised tiles ahead of the MMA.
-void pick_rings(int bt_cta, int r_pad, int &sx, int &sa, int &sc) {
+// dequantised tiles ahead of the MMA. A pair's K-step is twice as long and its
+// dequantised tiles cross the pair before the MMA can use them, so it keeps
+// more of them in flight and fewer activation stages.
+void pick_rings(int bt_cta, int r_pad, bool pair, int &sx, int &sa, int &sc) {
   const size_t budget = 227 * 1024;
+  if (pair) {
+    sx = kPairRings[0];
+    sa = kPairRings[1];
+    sc = kPairRings[2];
+    if (smem_bytes(bt_cta, r_pad, sx, sa, sc) <= budget) return;
+  }
   for (sx = 8; sx >= 4; --sx) {
     for (sc = 6; sc >= 4; sc -= 2) {
       sa = 3;
@@ -831,7 +885,23 @@ int token_tile(int64_t M) {
   if (M <= 128) return 128;
   return 256;
 }
+
+constexpr int kPairTokens = 512;   // token tile of a CTA pair (two N = 256 MMAs)
+
+// The CTA pair runs the linear forward and dX only. On B200 it measured no
+// faster than single-CTA tiles at the shapes of the 7B / 8B linears (the
+// kernel's K-step time grew with the pair's doubled MMA work instead of
+// staying at the dequantisation-bound single-CTA time), so the automatic
+// schedule keeps single CTAs and the pair runs when it is asked for.
+bool use_pair(const GemmArgs &a) {
+  return gemm_schedule() == 2 && a.mode <= 1 && a.M > 0;
+}
+
+std::atomic<int> g_schedule{0};
 }  // namespace
+
+void set_gemm_schedule(int schedule) { g_schedule.store(schedule, std::memory_order_relaxed); }
+int gemm_schedule() { return g_schedule.load(std::memory_order_relaxed); }
 
 size_t fused_gemm_ws_bytes(int64_t M) {
   const size_t sms = static_cast<size_t>(device_sm_count());
@@ -849,17 +919,15 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   p.M = a.M;
   p.mode = a.mode;
   const int bt = token_tile(a.M);
-  // The CTA-pair variant is compiled but not dispatched: on B200 its remote
-  // barrier arrivals cost more than the shared-memory traffic it saves.
-  const bool pair = false;
-  p.bt = bt;
-  p.bt_cta = pair ? bt / 2 : bt;
+  const bool pair = use_pair(a);
+  p.bt = pair ? kPairTokens : bt;
+  p.bt_cta = pair ? kPairTokens / 2 : bt;
   p.r_pad = a.r <= 16 ? 16 : (a.r <= 32 ? 32 : 64);
-  pick_rings(p.bt_cta, p.r_pad, p.sx, p.sa, p.sc);
+  pick_rings(p.bt_cta, p.r_pad, pair, p.sx, p.sa, p.sc);
   const int64_t rows = a.mode == 1 ? a.K : a.N;         // weight extent along UMMA M
   const int rows_per_tile = pair ? 2 * kTileRows : kTileRows;
   p.row_tiles = static_cast<int>((rows + rows_per_tile - 1) / rows_per_tile);
-  p.tok_tiles = static_cast<int>((a.M + bt - 1) / bt);
+  p.tok_tiles = static_cast<int>((a.M + p.bt - 1) / p.bt);
   p.nk = static_cast<int>(a.mode != 1 ? a.K / kKStage : (a.N + kKStage - 1) / kKStage);
 
   CUtensorMap tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux;
@@ -934,7 +1002,6 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
       default: return cudaErrorInvalidValue;
     }
   }
-  if (a.mode > 1) return cudaErrorInvalidValue;
   const void *pair_fn = a.mode == 0 ? reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true, 0, false>)
                                     : reinterpret_cast<const void *>(fused_nf4_gemm_kernel<true, 1, false>);
   cudaError_t e = cudaFuncSetAttribute(pair_fn, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -92,4 +92,8 @@ size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
 
 int device_sm_count();
 
+// Fused-GEMM tile schedule (qlora_schedule_t values), process-wide.
+void set_gemm_schedule(int schedule);
+int gemm_schedule();
+
 }  // namespace qlora

@@ -329,6 +329,23 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const uint16_t *X,
                                         uint16_t *Y, uint16_t *sU_out, int32_t *dev_status,
                                         qlora_stream_t stream);
 
+/*
+ * Tile schedule of the fused GEMM (qlora_fused_fwd, qlora_fused_dx and the
+ * composite calls that run them). Every schedule computes the same result up to
+ * fp32 summation order; this is a tuning and testing control.
+ *   QLORA_SCHEDULE_AUTO   the library's choice (default): single-CTA tiles of
+ *                         128 weight rows, stream-K for short token tiles
+ *   QLORA_SCHEDULE_SINGLE single-CTA tiles only
+ *   QLORA_SCHEDULE_PAIR   CTA pairs (cta_group::2, 256 weight rows x 512 tokens
+ *                         per pair tile) for the linear forward and dX; the
+ *                         SwiGLU modes keep single-CTA tiles
+ * The setting is process-wide and is read when a call launches its kernel; set
+ * it before launching (not while other host threads launch). Errors:
+ * INVALID_ARG for an unknown value.
+ */
+typedef enum { QLORA_SCHEDULE_AUTO = 0, QLORA_SCHEDULE_SINGLE = 1, QLORA_SCHEDULE_PAIR = 2 } qlora_schedule_t;
+qlora_status_t qlora_set_gemm_schedule(int32_t schedule);
+
 /* A static, human-readable name for a status code (host). */
 const char *qlora_status_string(qlora_status_t status);
 

@@ -113,3 +113,16 @@ def test_workspace_grows_with_tokens(lib):
     small = lib.linear_workspace(64, 1024, 1024, 8)
     big = lib.linear_workspace(2048, 4096, 4096, 16)
     assert 0 < small < big
+
+
+def test_gemm_schedule_control(lib):
+    """qlora_set_gemm_schedule accepts the three documented values and rejects
+    anything else with INVALID_ARG (a host-only call)."""
+    so = lib.library()
+    for v in (lib.SCHEDULE_SINGLE, lib.SCHEDULE_PAIR, lib.SCHEDULE_AUTO):
+        assert so.qlora_set_gemm_schedule(v) == 0
+    for v in (-1, 3, 1 << 20):
+        assert so.qlora_set_gemm_schedule(v) == 1
+    with lib.gemm_schedule(lib.SCHEDULE_PAIR):
+        pass
+    assert so.qlora_set_gemm_schedule(lib.SCHEDULE_AUTO) == 0

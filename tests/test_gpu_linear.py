@@ -125,7 +125,11 @@ def test_no_timeout_status(lib):
 SCHEDULE_CASES = [
     # N, K, M, r
     (2048, 1024, 300, 16),    # whole tiles: 32 FWD tiles of 16 K-steps
-    (2560, 256, 4000, 16),    # whole tiles: 320 FWD tiles, a ragged second wave
+    (2560, 256, 4000, 16),    # whole tiles: 320 FWD tiles, a ragged second wave; pairs: 80 FWD
+                              # pair tiles of 256 rows x 512 tokens, ragged last token tile
+    (4032, 512, 1100, 8),     # pairs: the last FWD pair tile's odd CTA holds 64 rows
+    (512, 4096, 1100, 32),    # pairs: 16 DX pair tiles of 256 dX columns, rank 32
+    (256, 4608, 1500, 64),    # pairs: rank 64 (the LoRA slices at 128-row offsets)
     (4096, 512, 8, 16),       # stream-K: each tile cut between about five CTAs
     (512, 4096, 64, 16),      # stream-K: 4 FWD tiles of 64 K-steps, ~37 CTAs per tile, more
                               # partials than fit in shared memory
@@ -136,8 +140,9 @@ SCHEDULE_CASES = [
 @pytest.mark.parametrize("N,K,M,r", SCHEDULE_CASES)
 def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
     """qlora_fused_fwd / qlora_fused_dx without a workspace (whole tiles per
-    CTA) and with one (stream-K, partial tiles summed through the workspace)
-    both match the oracle; the two differ only in fp32 summation order."""
+    CTA), with one (stream-K, partial tiles summed through the workspace) and
+    on CTA pairs (cta_group::2, selected with qlora_set_gemm_schedule) all
+    match the oracle; they differ only in fp32 summation order."""
     import torch
     s = 2.0
     h, d = _setup(lib, N, K, M, r, index=5)
@@ -151,11 +156,13 @@ def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
     gws = torch.full((lib.fused_workspace(M),), 0xAB, dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = {}
-    for name, ws in (("whole", None), ("streamk", gws)):
+    for name, ws, schedule in (("whole", None, lib.SCHEDULE_AUTO), ("streamk", gws, lib.SCHEDULE_AUTO),
+                               ("pair", None, lib.SCHEDULE_PAIR)):
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         dX = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda")
-        lib.fused_fwd(d["q"], d["X"], d["B"], sU, Y, status=st, ws=ws)
-        lib.fused_dx(d["q"], d["dY"], d["A"], sT, dX, status=st, ws=ws)
+        with lib.gemm_schedule(schedule):
+            lib.fused_fwd(d["q"], d["X"], d["B"], sU, Y, status=st, ws=ws)
+            lib.fused_dx(d["q"], d["dY"], d["A"], sT, dX, status=st, ws=ws)
         out[name] = (Y, dX)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
