@@ -277,6 +277,35 @@ def eight_b_set(q, torch):
     return mats
 
 
+def bench_quantize(q, torch, steps, warmup):
+    """a1-a3 (blockwise absmax, NF4 encode + pack, double quantisation) from
+    fp32 weights resident in HBM, over the seven linears of one 8B layer
+    (218 M weights); algorithmic bytes: 4 B read + 0.516 B written per weight."""
+    from bit_nf4_quantized_dequant_b200 import inputs
+    wl = inputs.WORKLOADS["set_8b"]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4040)
+    layer = wl.linears[:len({lin.name for lin in wl.linears})]
+    Ws = [torch.randn((lin.N, lin.K), generator=g, device="cuda", dtype=torch.float32) * 0.02 for lin in layer]
+    outs = [q.nf4_quantize(W) for W in Ws]
+    moved = sum(lin.N * lin.K * 4 + sum(q.nf4_sizes(lin.N, lin.K)) for lin in layer)
+    for _ in range(warmup):
+        for W, o in zip(Ws, outs):
+            q.nf4_quantize(W, out=o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        for W, o in zip(Ws, outs):
+            q.nf4_quantize(W, out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del Ws, outs
+    return {"workload": "quantize fp32 -> NF4 + double quant: the 7 linears of one set_8b layer",
+            "GB/s": moved / ms / 1e6, "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(layer)}
+
+
 def bench_dequant(q, torch, mats, steps, warmup):
     outs = [torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device="cuda") for lin, _ in mats]
     moved = sum(lin.N * lin.K * 2 + sum(q.nf4_sizes(lin.N, lin.K)) for lin, _ in mats)
@@ -394,15 +423,19 @@ def bench_decode(q, torch, mats, steps, warmup):
 
 
 def codec_error(q, torch):
-    """RMSE of NF4 and of the evenly spaced int4 comparison codebook (same
-    format) on the attention-projection weight, through the GPU codecs."""
+    """RMSE of NF4, of the evenly spaced int4 comparison codebook (same
+    format) and of NF4 with the fp8 mean-centred second level, on the
+    attention-projection weight, through the GPU codecs."""
     from bit_nf4_quantized_dequant_b200 import inputs
     W = torch.from_numpy(inputs.weight_f32(4096, 4096, index=0, outliers=True)).cuda()
     out = {"workload": "attn_proj_7b weight 4096x4096, N(0, 0.02) with 0.1% x8 outliers"}
     for name, book in (("nf4", q.CODEBOOK_NF4), ("int4", q.CODEBOOK_INT4)):
         back = q.codec_dequantize(q.codec_quantize(W, book), book).float()
         out[f"rmse_{name}"] = torch.sqrt(torch.mean((back - W) ** 2)).item()
+    back = q.dqfp8_dequantize(q.dqfp8_quantize(W)).float()
+    out["rmse_nf4_fp8_second_level"] = torch.sqrt(torch.mean((back - W) ** 2)).item()
     out["nf4_over_int4"] = out["rmse_nf4"] / out["rmse_int4"]
+    out["fp8_over_linear_second_level"] = out["rmse_nf4_fp8_second_level"] / out["rmse_nf4"]
     return out
 
 
@@ -717,6 +750,9 @@ def main():
     extras = {}
     if not args.no_extras:
         del sets
+        torch.cuda.empty_cache()
+        extras["quantize"] = bench_quantize(q, torch, steps=5, warmup=2)
+        extras["quantize"]["frac_of_hbm"] = extras["quantize"]["GB/s"] / peaks.get("hbm_gbs", 6650.0)
         torch.cuda.empty_cache()
         mats = eight_b_set(q, torch)
         extras["dequant"] = bench_dequant(q, torch, mats, steps=5, warmup=2)

@@ -21,7 +21,7 @@ __all__ = [
     "fused_workspace", "swiglu_fwd", "swiglu_bwd", "swiglu_pack_b", "swiglu_unpack_db", "swiglu_interleave",
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "adamw8_step", "AdamW8State", "set_gemm_schedule", "gemm_schedule",
-    "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR",
+    "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR", "dqfp8_sizes", "dqfp8_quantize", "dqfp8_dequantize",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -42,6 +42,7 @@ SYMBOLS = [
     "qlora_swiglu_fwd", "qlora_swiglu_bwd", "qlora_swiglu_pack_b", "qlora_swiglu_unpack_db",
     "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
     "qlora_adamw8_step", "qlora_set_gemm_schedule",
+    "qlora_dqfp8_sizes", "qlora_dqfp8_quantize", "qlora_dqfp8_dequantize",
 ]
 
 
@@ -111,6 +112,12 @@ def library():
     lib.qlora_adamw8_step.restype = st
     lib.qlora_set_gemm_schedule.argtypes = [ctypes.c_int32]
     lib.qlora_set_gemm_schedule.restype = st
+    lib.qlora_dqfp8_sizes.argtypes = [_I64, _I64, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]
+    lib.qlora_dqfp8_sizes.restype = st
+    lib.qlora_dqfp8_quantize.argtypes = [_P, ctypes.POINTER(_NF4), _P, _P]
+    lib.qlora_dqfp8_quantize.restype = st
+    lib.qlora_dqfp8_dequantize.argtypes = [ctypes.POINTER(_NF4), _P, _P]
+    lib.qlora_dqfp8_dequantize.restype = st
     lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_codec_levels.restype = st
     lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
@@ -480,3 +487,37 @@ class gemm_schedule:
 
 def set_gemm_schedule(schedule: int) -> None:
     _check(library().qlora_set_gemm_schedule(int(schedule)), "qlora_set_gemm_schedule")
+
+
+# ---------------------------------------------------------------------------
+# comparison second level: E4M3 codes of mean-centred block constants
+# ---------------------------------------------------------------------------
+def dqfp8_sizes(rows: int, cols: int):
+    a, b, c = _SZ(), _SZ(), _SZ()
+    _check(library().qlora_dqfp8_sizes(rows, cols, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "qlora_dqfp8_sizes")
+    return a.value, b.value, c.value
+
+
+def dqfp8_quantize(W, status=None, stream=None) -> NF4Matrix:
+    """NF4 codes with the fp8 mean-centred second level; scale2 holds (d, mu)
+    per group of 256 blocks."""
+    import torch
+    rows, cols = W.shape
+    cb, sb, s2b = dqfp8_sizes(rows, cols)
+    q = NF4Matrix(rows, cols, torch.empty(cb, dtype=torch.uint8, device=W.device),
+                  torch.empty(sb, dtype=torch.uint8, device=W.device),
+                  torch.empty(s2b // 4, dtype=torch.float32, device=W.device))
+    s = q.c_struct()
+    _check(library().qlora_dqfp8_quantize(_ptr(W), ctypes.byref(s), _ptr(status), _stream(stream)),
+           "qlora_dqfp8_quantize")
+    return q
+
+
+def dqfp8_dequantize(q: NF4Matrix, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.codes.device)
+    s = q.c_struct()
+    _check(library().qlora_dqfp8_dequantize(ctypes.byref(s), _ptr(out), _stream(stream)), "qlora_dqfp8_dequantize")
+    return out

@@ -198,6 +198,34 @@ qlora_status_t qlora_codec_dequantize(const qlora_nf4_t *q, int32_t codebook, ui
                                        reinterpret_cast<cudaStream_t>(stream), codebook));
 }
 
+qlora_status_t qlora_dqfp8_sizes(int64_t rows, int64_t cols, size_t *codes_b, size_t *s8_b, size_t *s2_b) {
+  qlora_status_t st = qlora_nf4_sizes(rows, cols, codes_b, s8_b, s2_b);
+  if (st == QLORA_OK && s2_b) *s2_b *= 2;   // (d, mu) per group
+  return st;
+}
+
+qlora_status_t qlora_dqfp8_quantize(const float *W, const qlora_nf4_t *q, int32_t *dev_status,
+                                    qlora_stream_t stream) {
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(q->scale2) & 7u) return QLORA_ERR_MISALIGNED;
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_quantize(W, q->rows, q->cols, q->codes, q->scale8, q->scale2, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream), QLORA_CODEBOOK_NF4, 1));
+}
+
+qlora_status_t qlora_dqfp8_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora_stream_t stream) {
+  qlora_status_t st = check_nf4(q);
+  if (st != QLORA_OK) return st;
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(out)) return QLORA_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(q->scale2) & 7u) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_dequantize(q->codes, q->scale8, q->scale2, q->rows, q->cols, out,
+                                       reinterpret_cast<cudaStream_t>(stream), QLORA_CODEBOOK_NF4, 1));
+}
+
 qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t *bytes) {
   if (!bytes || M <= 0 || N <= 0 || K <= 0) return QLORA_ERR_INVALID_ARG;
   if (K % kBlock || N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;

@@ -5,10 +5,36 @@
 // QLoRA ...", section "The three QLoRA ideas"): blocks of 64 consecutive
 // row-major weights, 4-bit codes into the NF4 levels, one 8-bit constant per
 // block, one fp32 second-level scale per group of 256 blocks.
+#include <cuda_fp8.h>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
 namespace {
+
+// Second-level formats: kDqLinear = unsigned linear absmax codes, one fp32
+// scale per group (the library's format); kDqFp8 = E4M3 codes of the
+// group-mean-centred constants, fp32 (d, mu) per group (the comparison
+// format of the paper the pages cite: "QLoRA and Fine-Tuning on One Consumer
+// GPU", "NF4 and double quantisation"). Decoded constant for kDqFp8:
+// s = RN32(RN32(e4m3(q) * d) + mu).
+constexpr int kDqLinear = 0;
+constexpr int kDqFp8 = 1;
+constexpr float kE4m3Max = 448.0f;
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t q) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3)));
+}
+
+template <int DQ>
+__device__ __forceinline__ float decoded_scale(const uint8_t *scale8, const float *scale2, int64_t b) {
+  if constexpr (DQ == kDqFp8) {
+    const float2 dm = __ldg(reinterpret_cast<const float2 *>(scale2) + (b >> 8));
+    return __fadd_rn(__fmul_rn(e4m3_to_float(__ldg(scale8 + b)), dm.x), dm.y);
+  } else {
+    return block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
+  }
+}
 
 // code = number of midpoints between adjacent levels that n lies strictly
 // above: the nearest level, ties to the lower one. The midpoints of two float32
@@ -28,10 +54,13 @@ __device__ __forceinline__ uint32_t nearest_level(float n) {
   return code;
 }
 
-// One CTA per group of 256 blocks; warp w handles blocks w, w+8, ...; lane l
-// holds elements 2l and 2l+1 of a block, so the packed byte l of the block is
+// One CTA per group of 256 blocks; warp w handles blocks w, w+8, ..., four at
+// a time (four independent 256-byte loads in flight per warp); lane l holds
+// elements 2l and 2l+1 of a block, so the packed byte l of the block is
 // written by lane l.
-template <int BOOK>
+constexpr int kQuantBatch = 4;
+
+template <int BOOK, int DQ>
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restrict__ W, int64_t nb,
                                                            uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scale8,
@@ -39,6 +68,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
                                                            int32_t *status) {
   __shared__ float c1s[kGroup];
   __shared__ float red[8];
+  __shared__ float mu_s;
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * kGroup;
   const int nblk = static_cast<int>(nb - b0 < kGroup ? nb - b0 : kGroup);
@@ -46,28 +76,66 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
   const int lane = threadIdx.x & 31;
 
   bool bad = false;
-  for (int i = warp; i < nblk; i += 8) {
-    const int64_t b = b0 + i;
-    const float2 v = __ldg(reinterpret_cast<const float2 *>(W + b * kBlock) + lane);
-    bad |= !isfinite(v.x) || !isfinite(v.y);
-    float m = fmaxf(fabsf(v.x), fabsf(v.y));
+  for (int i0 = warp; i0 < nblk; i0 += 8 * kQuantBatch) {
+    float2 v[kQuantBatch];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    constexpr uint32_t kZero = BOOK == kBookInt4 ? 8u : 7u;   // index of the exact zero level
-    uint32_t e0 = kZero, e1 = kZero;
-    if (m > 0.f) {
-      e0 = nearest_level<BOOK>(__fdiv_rn(v.x, m));
-      e1 = nearest_level<BOOK>(__fdiv_rn(v.y, m));
+    for (int u = 0; u < kQuantBatch; ++u) {   // warp-uniform guard: the block exists or not
+      const int i = i0 + 8 * u;
+      v[u] = i < nblk ? __ldg(reinterpret_cast<const float2 *>(W + (b0 + i) * kBlock) + lane) : make_float2(0.f, 0.f);
     }
-    codes[b * (kBlock / 2) + lane] = static_cast<uint8_t>((e0 << 4) | e1);
-    if (lane == 0) c1s[i] = m;
+#pragma unroll
+    for (int u = 0; u < kQuantBatch; ++u) {
+      const int i = i0 + 8 * u;
+      if (i >= nblk) break;
+      const int64_t b = b0 + i;
+      bad |= !isfinite(v[u].x) || !isfinite(v[u].y);
+      float m = fmaxf(fabsf(v[u].x), fabsf(v[u].y));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      constexpr uint32_t kZero = BOOK == kBookInt4 ? 8u : 7u;   // index of the exact zero level
+      uint32_t e0 = kZero, e1 = kZero;
+      if (m > 0.f) {
+        e0 = nearest_level<BOOK>(__fdiv_rn(v[u].x, m));
+        e1 = nearest_level<BOOK>(__fdiv_rn(v[u].y, m));
+      }
+      codes[b * (kBlock / 2) + lane] = static_cast<uint8_t>((e0 << 4) | e1);
+      if (lane == 0) c1s[i] = m;
+    }
   }
   if (bad) set_status(status, 5 /* QLORA_ERR_NONFINITE */);
   __syncthreads();
 
-  // second level: c2 = max c1 over the group
   const int t = threadIdx.x;
   const float c1 = t < nblk ? c1s[t] : 0.f;
+  if constexpr (DQ == kDqFp8) {
+    // mean of the group's constants: float64 sum in block order, one division
+    if (t == 0) {
+      double sum = 0.0;
+      for (int i = 0; i < nblk; ++i) sum = __dadd_rn(sum, static_cast<double>(c1s[i]));
+      mu_s = __double2float_rn(__ddiv_rn(sum, static_cast<double>(nblk)));
+    }
+    __syncthreads();
+    const float mu = mu_s;
+    const float cen = t < nblk ? __fsub_rn(c1, mu) : 0.f;
+    float a = fabsf(cen);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    float amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float d = __fdiv_rn(amax, kE4m3Max);
+    if (t < nblk)
+      scale8[b0 + t] = d > 0.f ? static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(cen, d), __NV_SATFINITE, __NV_E4M3))
+                               : uint8_t{0};
+    if (t == 0) {
+      scale2[2 * g] = d;
+      scale2[2 * g + 1] = mu;
+    }
+    return;
+  }
+  // second level: c2 = max c1 over the group
   float m = c1;
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -93,7 +161,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
 // Each warp stages its 32 x 64 contiguous output bytes in shared memory and
 // writes them with one bulk copy, so global stores are full, contiguous 2 KiB
 // runs instead of 64-byte pieces strided across the warp.
-template <int BOOK>
+template <int BOOK, int DQ>
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
                                                           const uint8_t *__restrict__ scale8,
                                                           const float *__restrict__ scale2,
@@ -108,7 +176,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
   if (i < nhalf) {
     const int64_t b = i >> 1;
     const uint4 c = __ldg(reinterpret_cast<const uint4 *>(codes) + i);
-    const float sc = block_scale(__ldg(scale8 + b), __ldg(scale2 + (b >> 8)));
+    const float sc = decoded_scale<DQ>(scale8, scale2, b);
     const Nf4Table t = make_table_book<BOOK>(sc);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -131,28 +199,34 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
-                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book) {
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book, int dq) {
   const int64_t nb = rows * cols / kBlock;
   const int64_t ng = (nb + kGroup - 1) / kGroup;
   if (dev_status) {
     cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
   }
-  if (book == kBookInt4)
-    nf4_quantize_kernel<kBookInt4><<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+  const unsigned grid = static_cast<unsigned>(ng);
+  if (dq == kDqFp8)
+    nf4_quantize_kernel<kBookNf4, kDqFp8><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+  else if (book == kBookInt4)
+    nf4_quantize_kernel<kBookInt4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
   else
-    nf4_quantize_kernel<kBookNf4><<<static_cast<unsigned>(ng), 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+    nf4_quantize_kernel<kBookNf4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
-                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book) {
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book, int dq) {
   const int64_t nhalf = rows * cols / 32;
   const int64_t grid = (nhalf + 255) / 256;
-  if (book == kBookInt4)
-    nf4_dequant_kernel<kBookInt4><<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (dq == kDqFp8)
+    nf4_dequant_kernel<kBookNf4, kDqFp8><<<g, 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+  else if (book == kBookInt4)
+    nf4_dequant_kernel<kBookInt4, kDqLinear><<<g, 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
   else
-    nf4_dequant_kernel<kBookNf4><<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
+    nf4_dequant_kernel<kBookNf4, kDqLinear><<<g, 256, 0, s>>>(codes, scale8, scale2, nhalf, out);
   return cudaGetLastError();
 }
 

@@ -12,10 +12,13 @@ constexpr int kGroup = 256;   // blocks per second-level group
 
 // Kernel launchers. Each returns the cudaError_t of the launch.
 // book: 0 = NF4, 1 = the evenly spaced int4 comparison codebook.
+// dq: 0 = linear 8-bit second level (scale2: one float per group), 1 = E4M3
+// codes of mean-centred constants (scale2: d, mu per group; NF4 book only).
 cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t *codes,
-                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book = 0);
+                            uint8_t *scale8, float *scale2, int32_t *dev_status, cudaStream_t s, int book = 0,
+                            int dq = 0);
 cudaError_t launch_dequantize(const uint8_t *codes, const uint8_t *scale8, const float *scale2,
-                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book = 0);
+                              int64_t rows, int64_t cols, uint16_t *out, cudaStream_t s, int book = 0, int dq = 0);
 
 // Fused NF4 GEMM (tcgen05). Mode FWD: Y[M,N] = X[M,K] W'^T + sU[M,r] Bl^T.
 // Mode DX: dX[M,K] = dY[M,N] W' + sT[M,r] Al.

@@ -121,6 +121,32 @@ qlora_status_t qlora_codec_quantize(const float *W, const qlora_nf4_t *q, int32_
                                     qlora_stream_t stream);
 qlora_status_t qlora_codec_dequantize(const qlora_nf4_t *q, int32_t codebook, uint16_t *out, qlora_stream_t stream);
 
+/* Comparison second level. NF4 codes and first-level blocks as above, with
+ * the block constants stored the way the paper the pages cite does it
+ * ("QLoRA and Fine-Tuning on One Consumer GPU", "NF4 and double
+ * quantisation": double quantisation quantises the absmax constants and saves
+ * about 0.37 bits per parameter; "What is QLoRA ...", "The three QLoRA ideas":
+ * 8 bits in blocks of 256): per group of 256 blocks the constants are centred
+ * on their mean and kept as 8-bit floats.
+ *   mu_g = RN32(RN64(S / n)), S the float64 sum of the group's c1_b in block
+ *          order, n its blocks; cen_b = RN32(c1_b - mu_g); a_g = max |cen_b|;
+ *   d_g = RN32(a_g / 448); scale8[b] = E4M3 code of RN32(cen_b / d_g)
+ *          (round to nearest even, saturating to +-448; 0 when d_g = 0);
+ *   scale2[2g] = d_g, scale2[2g + 1] = mu_g (2 * ng floats, 8-byte aligned);
+ *   block scale s_b = RN32(RN32(e4m3(scale8[b]) * d_g) + mu_g) and
+ *   w' = RN_bf16(RN32(level[code] * s_b)).
+ * 4 + 8/64 + 64/16384 = 4.1289 bits per weight. Only the codec runs on this
+ * format (the GEMMs read the linear one); it exists to measure the error of
+ * the two second levels on the same weights.
+ * qlora_dqfp8_sizes: as qlora_nf4_sizes with s2_b = 8 * ng. Errors: INVALID_ARG.
+ * qlora_dqfp8_quantize / qlora_dqfp8_dequantize: as qlora_nf4_quantize /
+ * qlora_nf4_dequantize. Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED,
+ * CUDA; NONFINITE in dev_status. */
+qlora_status_t qlora_dqfp8_sizes(int64_t rows, int64_t cols, size_t *codes_b, size_t *s8_b, size_t *s2_b);
+qlora_status_t qlora_dqfp8_quantize(const float *W, const qlora_nf4_t *q, int32_t *dev_status,
+                                    qlora_stream_t stream);
+qlora_status_t qlora_dqfp8_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora_stream_t stream);
+
 /* Workspace bytes that qlora_linear_fwd and qlora_linear_bwd need for M
  * tokens through an [N, K] layer of rank r (host). The same workspace may be
  * reused by consecutive calls on one stream; calls that run concurrently need

@@ -121,3 +121,53 @@ def test_nf4_error_below_int4_on_the_gpu(lib):
         back = lib.codec_dequantize(lib.codec_quantize(W, book), book).float()
         err[book] = torch.sqrt(torch.mean((back - W) ** 2)).item()
     assert err[lib.CODEBOOK_NF4] < 0.9 * err[lib.CODEBOOK_INT4]
+
+
+def _fp8dq_case(kind):
+    g = inputs.rng(40)
+    if kind == "ragged":            # 240 blocks: one short group
+        return (g.standard_normal((48, 320)) * 0.02).astype(np.float32)
+    if kind == "constant":          # every block's absmax 0.03: d = 0, codes +0
+        W = (g.uniform(-0.03, 0.03, (64, 512))).astype(np.float32)
+        W.reshape(-1, 64)[:, 5] = 0.03
+        return W
+    if kind == "zeros":             # all-zero blocks inside groups of non-zero ones
+        W = (g.standard_normal((256, 1024)) * 0.02).astype(np.float32)
+        W[7, :] = 0.0
+        W[100, 64:192] = 0.0
+        return W
+    return inputs.weight_f32(1024, 4096, index=9, outliers=True)
+
+
+@pytest.mark.parametrize("kind", ["outliers", "ragged", "constant", "zeros"])
+def test_fp8_second_level_bit_exact(lib, kind):
+    """The comparison second level (E4M3 codes of mean-centred block
+    constants, (d, mu) per group): codes, E4M3 codes, the float32 pairs and
+    the dequantised bf16 weight bit for bit against oracle.dq_fp8."""
+    import torch
+    from oracle import dq_fp8
+    W = _fp8dq_case(kind)
+    N, K = W.shape
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = lib.dqfp8_quantize(torch.from_numpy(W).cuda(), status=st)
+    out = lib.dqfp8_dequantize(q)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    p, s8, s2 = dq_fp8.quantize_fp8dq(W)
+    np.testing.assert_array_equal(q.codes.cpu().numpy(), p)
+    np.testing.assert_array_equal(q.scale8.cpu().numpy(), s8)
+    np.testing.assert_array_equal(q.scale2.cpu().numpy().view(np.uint32), s2.reshape(-1).view(np.uint32))
+    np.testing.assert_array_equal(bf16_dev_bits(out), dq_fp8.dequantize_fp8dq_bits(p, s8, s2, N, K))
+
+
+def test_fp8_and_linear_second_levels_err_alike(lib):
+    """Both second levels on the same 4096 x 4096 weight (N(0, 0.02), 0.1 %
+    x8 outliers): the dequantisation error of the two differs by a few
+    percent at most, since both keep the block constants to about 8 bits."""
+    import torch
+    W = torch.from_numpy(inputs.weight_f32(4096, 4096, index=8, outliers=True)).cuda()
+    lin = lib.nf4_dequantize(lib.nf4_quantize(W)).float()
+    f8 = lib.dqfp8_dequantize(lib.dqfp8_quantize(W)).float()
+    e_lin = torch.sqrt(torch.mean((lin - W) ** 2)).item()
+    e_f8 = torch.sqrt(torch.mean((f8 - W) ** 2)).item()
+    assert abs(e_f8 - e_lin) < 0.03 * e_lin
