@@ -22,6 +22,7 @@ __all__ = [
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "adamw8_step", "AdamW8State", "set_gemm_schedule", "gemm_schedule",
     "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR", "dqfp8_sizes", "dqfp8_quantize", "dqfp8_dequantize",
+    "lora_grads_adamw8",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +44,13 @@ SYMBOLS = [
     "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
     "qlora_adamw8_step", "qlora_set_gemm_schedule",
     "qlora_dqfp8_sizes", "qlora_dqfp8_quantize", "qlora_dqfp8_dequantize",
+    "qlora_lora_grads_adamw8",
 ]
+
+
+class _Adam8(ctypes.Structure):
+    _fields_ = [("p", ctypes.c_void_p), ("p_bf16", ctypes.c_void_p), ("m_q", ctypes.c_void_p),
+                ("v_q", ctypes.c_void_p), ("m_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p)]
 
 
 class QloraUnavailable(RuntimeError):
@@ -118,6 +125,11 @@ def library():
     lib.qlora_dqfp8_quantize.restype = st
     lib.qlora_dqfp8_dequantize.argtypes = [ctypes.POINTER(_NF4), _P, _P]
     lib.qlora_dqfp8_dequantize.restype = st
+    lib.qlora_lora_grads_adamw8.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_int32, _P, _P,
+                                            ctypes.POINTER(_Adam8), ctypes.POINTER(_Adam8), ctypes.c_int32,
+                                            ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                            ctypes.c_float, _P]
+    lib.qlora_lora_grads_adamw8.restype = st
     lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_codec_levels.restype = st
     lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
@@ -521,3 +533,26 @@ def dqfp8_dequantize(q: NF4Matrix, out=None, stream=None):
     s = q.c_struct()
     _check(library().qlora_dqfp8_dequantize(ctypes.byref(s), _ptr(out), _stream(stream)), "qlora_dqfp8_dequantize")
     return out
+
+
+def lora_grads_adamw8(X, dY, sU, sT, A_master, B_master, A_state: AdamW8State, B_state: AdamW8State, lr: float,
+                      beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                      A_bf16=None, B_bf16=None, dA=None, dB=None, stream=None):
+    """Adapter gradients and one 8-bit AdamW step of both adapters in one
+    launch (qlora_lora_grads_adamw8). A_master is the fp32 master copy of A^T
+    ([K, r]), B_master that of B ([N, r]); A_bf16 [r, K] and B_bf16 [N, r]
+    receive the bf16 operands; dA [r, K] / dB [N, r] the fp32 gradients when
+    given. Both states advance one step (they share the step count)."""
+    M, K = X.shape
+    N = dY.shape[1]
+    r = sU.shape[1]
+    A_state.step += 1
+    B_state.step = A_state.step
+    ptr = lambda t: None if t is None else t.data_ptr()
+    a = _Adam8(A_master.data_ptr(), ptr(A_bf16), A_state.m_q.data_ptr(), A_state.v_q.data_ptr(),
+               A_state.m_scale.data_ptr(), A_state.v_scale.data_ptr())
+    b = _Adam8(B_master.data_ptr(), ptr(B_bf16), B_state.m_q.data_ptr(), B_state.v_q.data_ptr(),
+               B_state.m_scale.data_ptr(), B_state.v_scale.data_ptr())
+    _check(library().qlora_lora_grads_adamw8(_ptr(X), _ptr(dY), M, N, K, _ptr(sU), _ptr(sT), r, _ptr(dA), _ptr(dB),
+                                             ctypes.byref(a), ctypes.byref(b), A_state.step, lr, beta1, beta2, eps,
+                                             weight_decay, _stream(stream)), "qlora_lora_grads_adamw8")

@@ -11,6 +11,7 @@
 
 #include "qlora.h"
 #include "qlora_device.cuh"
+#include "adamw8.cuh"
 #include "qlora_internal.h"
 
 namespace qlora {
@@ -316,6 +317,38 @@ qlora_status_t qlora_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M
   const size_t need = 4 * (fa > fb ? fa : fb);
   if (need > 0 && (!ws || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   return cuda_status(launch_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static bool adam_tensor_ok(const qlora_adamw8_tensor_t *t) {
+  return t && t->p && t->m_q && t->v_q && t->m_scale && t->v_scale;
+}
+
+qlora_status_t qlora_lora_grads_adamw8(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                                       const uint16_t *sU, const uint16_t *sT, int32_t r, float *dA, float *dB,
+                                       const qlora_adamw8_tensor_t *A_state, const qlora_adamw8_tensor_t *B_state,
+                                       int32_t step, float lr, float beta1, float beta2, float eps,
+                                       float weight_decay, qlora_stream_t stream) {
+  if (!X || !dY || !sU || !sT || M <= 0 || N <= 0 || K <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!adam_tensor_ok(A_state) || !adam_tensor_ok(B_state)) return QLORA_ERR_INVALID_ARG;
+  if (step < 1 || !std::isfinite(lr) || !(eps > 0.f) || !std::isfinite(weight_decay) ||
+      !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+    return QLORA_ERR_INVALID_ARG;
+  if (K % kBlock || N % 16 || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(dY) || !aligned16(sU) || !aligned16(sT) || (dA && !aligned16(dA)) ||
+      (dB && !aligned16(dB)))
+    return QLORA_ERR_MISALIGNED;
+  qlora::AdamFuseArgs a{};
+  a.A = {A_state->p, A_state->m_q, A_state->v_q, A_state->m_scale, A_state->v_scale};
+  a.B = {B_state->p, B_state->m_q, B_state->v_q, B_state->m_scale, B_state->v_scale};
+  a.A_bf16 = A_state->p_bf16;
+  a.B_bf16 = B_state->p_bf16;
+  a.step = step;
+  a.lr = lr;
+  a.beta1 = beta1;
+  a.beta2 = beta2;
+  a.eps = eps;
+  a.wd = weight_decay;
+  return cuda_status(launch_lora_grads(X, dY, M, N, K, sU, sT, r, dA, dB, reinterpret_cast<cudaStream_t>(stream), &a));
 }
 
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,

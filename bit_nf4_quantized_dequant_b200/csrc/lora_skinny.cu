@@ -13,6 +13,7 @@
 // the result is deterministic.
 #include <cuda.h>
 
+#include "adamw8.cuh"
 #include "qlora_device.cuh"
 
 namespace qlora {
@@ -182,17 +183,29 @@ __global__ void __launch_bounds__(160) lora_rows_kernel(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 struct ColsProblem {
   int64_t D;
-  float *out;
+  float *out;          // may be NULL when the gradients feed the fused AdamW step only
   int transpose_out;
 };
 
-template <int NT>
+// The 8-bit AdamW step fused into the epilogue. A CTA's tile holds the
+// gradients of 128 consecutive d for every j < r, so in the d-major order
+// (element d * r + j) it is r / 2 whole state blocks of 256: product 0's state
+// is kept for A^T (A's master copy flattened as [K, r]), product 1's for B
+// ([N, r], its natural order). bf16 copies go to A [r, K] and B [N, r], the
+// operands the kernels read.
+struct AdamFuse {
+  Adam8Tensor t[2];
+  uint16_t *bf16[2];
+  AdamArgs a;
+};
+
+template <int NT, bool kAdam>
 __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ CUtensorMap tm_z0,
                                                         const __grid_constant__ CUtensorMap tm_v0,
                                                         const __grid_constant__ CUtensorMap tm_z1,
                                                         const __grid_constant__ CUtensorMap tm_v1, ColsProblem p0,
                                                         ColsProblem p1, int tiles0, int64_t M, int r,
-                                                        int mb_per_cta, int32_t *status) {
+                                                        int mb_per_cta, int32_t *status, AdamFuse af) {
   constexpr int r_pad = NT * 8;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -302,10 +315,58 @@ __global__ void __launch_bounds__(288) lora_cols_kernel(const __grid_constant__ 
     }
   }
   cluster_sync_all();
+  const uint32_t red_addr = smem_u32(red);
+  if constexpr (kAdam) {
+    // whole state blocks, one warp each, spread over the cluster's CTAs; the
+    // gradient of each element is summed over the partials in rank order, as below
+    const int which = second ? 1 : 0;
+    const Adam8Tensor t = af.t[which];
+    uint16_t *const pb = af.bf16[which];
+    const int64_t n = pr.D * r;
+    const int tile_blocks = (128 * r) / kStateBlock;
+    const int64_t blk0 = d0 * r / kStateBlock;
+    const int nwarps = static_cast<int>(blockDim.x >> 5);
+    for (int bk = static_cast<int>(rank) * nwarps + warp; bk < tile_blocks; bk += csize * nwarps) {
+      const int64_t blk = blk0 + bk;
+      if (blk * kStateBlock >= n) break;
+      float g[8], pn[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int il = bk * kStateBlock + e * 32 + lane;
+        const int row = il / r, j = il % r;
+        const int64_t d = d0 + row;
+        g[e] = 0.f;
+        if (d < pr.D) {
+          const uint32_t off = static_cast<uint32_t>((row * r_pad + j) * 4);
+          float sum = 0.f;
+          for (int q = 0; q < csize; ++q) sum += ld_dsmem_f32(mapa_shared(red_addr + off, static_cast<uint32_t>(q)));
+          g[e] = sum;
+          if (pr.out) {
+            if (pr.transpose_out) pr.out[static_cast<int64_t>(j) * pr.D + d] = sum;
+            else                  pr.out[d * r + j] = sum;
+          }
+        }
+      }
+      adamw8_block(t, blk, n, g, af.a, pn);
+      if (pb) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int il = bk * kStateBlock + e * 32 + lane;
+          const int row = il / r, j = il % r;
+          const int64_t d = d0 + row;
+          if (d < pr.D) {
+            const int64_t o = which == 0 ? static_cast<int64_t>(j) * pr.D + d : d * r + j;
+            pb[o] = __bfloat16_as_ushort(__float2bfloat16_rn(pn[e]));
+          }
+        }
+      }
+    }
+    cluster_sync_all();
+    return;
+  }
   const int rows_per = (128 + csize - 1) / csize;
   const int r_lo = static_cast<int>(rank) * rows_per;
   const int r_hi = r_lo + rows_per < 128 ? r_lo + rows_per : 128;
-  const uint32_t red_addr = smem_u32(red);
   for (int e = threadIdx.x; e < (r_hi - r_lo) * r; e += blockDim.x) {
     const int row = r_lo + e / r, j = e % r;
     const int64_t d = d0 + row;
@@ -398,7 +459,8 @@ cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint
 }
 
 cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
-                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st) {
+                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st,
+                              const AdamFuseArgs *adam) {
   const int r_pad = pad_rank(r);
   CUtensorMap tz0, tv0, tz1, tv1;
   // product 0: dA[j, k] = sum_m sT[m, j] X[m, k]  (D = K, transposed output)
@@ -418,13 +480,24 @@ cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, 
   int64_t Mv = M;
   int rv = r;
   int32_t *status = nullptr;
-  void *args[] = {&tz0, &tv0, &tz1, &tv1, &p0, &p1, &t0v, &Mv, &rv, &mb_per_cta, &status};
+  AdamFuse af{};
+  if (adam) {
+    af.t[0] = adam->A;
+    af.t[1] = adam->B;
+    af.bf16[0] = adam->A_bf16;
+    af.bf16[1] = adam->B_bf16;
+    af.a = make_adam_args(adam->step, adam->lr, adam->beta1, adam->beta2, adam->eps, adam->wd);
+  }
+  void *args[] = {&tz0, &tv0, &tz1, &tv1, &p0, &p1, &t0v, &Mv, &rv, &mb_per_cta, &status, &af};
   const dim3 grid(static_cast<unsigned>(tiles0 + tiles1), static_cast<unsigned>(csize));
   const size_t smem = cols_smem(r_pad);
-  switch (r_pad / 8) {
-    case 2: return launch_cluster(lora_cols_kernel<2>, grid, 288, smem, st, csize, args);
-    case 4: return launch_cluster(lora_cols_kernel<4>, grid, 288, smem, st, csize, args);
-    case 8: return launch_cluster(lora_cols_kernel<8>, grid, 288, smem, st, csize, args);
+  switch ((r_pad / 8) * 2 + (adam ? 1 : 0)) {
+    case 4: return launch_cluster(lora_cols_kernel<2, false>, grid, 288, smem, st, csize, args);
+    case 5: return launch_cluster(lora_cols_kernel<2, true>, grid, 288, smem, st, csize, args);
+    case 8: return launch_cluster(lora_cols_kernel<4, false>, grid, 288, smem, st, csize, args);
+    case 9: return launch_cluster(lora_cols_kernel<4, true>, grid, 288, smem, st, csize, args);
+    case 16: return launch_cluster(lora_cols_kernel<8, false>, grid, 288, smem, st, csize, args);
+    case 17: return launch_cluster(lora_cols_kernel<8, true>, grid, 288, smem, st, csize, args);
     default: return cudaErrorInvalidValue;
   }
 }

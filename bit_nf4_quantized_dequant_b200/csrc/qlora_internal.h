@@ -88,8 +88,10 @@ cudaError_t launch_lora_rows(const uint16_t *Z, int64_t M, int64_t K, const uint
                              cudaStream_t st);
 // Adapter gradients in one launch: dA[j, k] = sum_m sT[m, j] X[m, k] and
 // dB[n, j] = sum_m dY[m, n] sU[m, j] (fp32, overwritten).
+struct AdamFuseArgs;
 cudaError_t launch_lora_grads(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
-                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st);
+                              const uint16_t *sU, const uint16_t *sT, int r, float *dA, float *dB, cudaStream_t st,
+                              const AdamFuseArgs *adam = nullptr);
 size_t lora_rows_ws_floats(int64_t M, int64_t K, int r);
 size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
 

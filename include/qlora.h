@@ -327,6 +327,35 @@ qlora_status_t qlora_adamw8_step(float *p, uint16_t *p_bf16, const float *grad, 
                                  float *m_scale, float *v_scale, int64_t n, int32_t step, float lr, float beta1,
                                  float beta2, float eps, float weight_decay, qlora_stream_t stream);
 
+/* The adapter gradients of qlora_lora_grads and, in the same launch, one
+ * qlora_adamw8_step of both adapters (the update fused into the gradient
+ * epilogue: each gradient tile covers whole 256-element state blocks, so no
+ * gradient needs to go through memory). The state of each adapter is kept in
+ * the order of its gradient tiles, d-major:
+ *   A: p[d * r + j] is A[j][d] (the master copy of A^T, [K, r] flattened),
+ *      and so are m_q, v_q (blocks of 256 in that order); p_bf16 is A itself,
+ *      [r, K] bf16, written transposed;
+ *   B: p[n * r + j] is B[n][j] ([N, r], natural order); p_bf16 is B [N, r].
+ * The result is bit for bit that of qlora_lora_grads followed by
+ * qlora_adamw8_step on dA^T (A) and dB (B) with these layouts. dA and dB are
+ * still written when not NULL (fp32, as qlora_lora_grads). The launch reads
+ * X, dY, sU and sT only, so A and B may be updated in place while sU, sT
+ * computed from them are its inputs.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA. */
+typedef struct {
+  float *p;
+  uint16_t *p_bf16;   /* may be NULL */
+  int8_t *m_q;
+  uint8_t *v_q;
+  float *m_scale;
+  float *v_scale;
+} qlora_adamw8_tensor_t;
+qlora_status_t qlora_lora_grads_adamw8(const uint16_t *X, const uint16_t *dY, int64_t M, int64_t N, int64_t K,
+                                       const uint16_t *sU, const uint16_t *sT, int32_t r, float *dA, float *dB,
+                                       const qlora_adamw8_tensor_t *A_state, const qlora_adamw8_tensor_t *B_state,
+                                       int32_t step, float lr, float beta1, float beta2, float eps,
+                                       float weight_decay, qlora_stream_t stream);
+
 /*
  * Allocation-free forward. The pages have no counterpart to this call: it is an
  * interface convenience of this library for callers that cannot allocate
