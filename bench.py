@@ -439,6 +439,47 @@ def codec_error(q, torch):
     return out
 
 
+def bench_adamw8(q, torch, steps, warmup):
+    """The adapter-gradient launch with the 8-bit AdamW step of A and B fused
+    into its epilogue, against the gradients followed by two standalone steps,
+    on the attention projection (4096 x 4096, 2048 tokens, r = 16)."""
+    M, N, K, r = 2048, 4096, 4096, 16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5151)
+    bf = lambda *shape: torch.randn(*shape, generator=g, device="cuda").bfloat16()
+    X, dY, sU, sT = bf(M, K), bf(M, N), bf(M, r), bf(M, r)
+    Am = torch.randn(K, r, generator=g, device="cuda") / r
+    Bm = torch.randn(N, r, generator=g, device="cuda") * 0.01
+    Ab, Bb = torch.empty(r, K, dtype=torch.bfloat16, device="cuda"), torch.empty(N, r, dtype=torch.bfloat16, device="cuda")
+    dA, dB = torch.empty(r, K, device="cuda"), torch.empty(N, r, device="cuda")
+    dAt = torch.empty(K, r, device="cuda")
+    ws = torch.empty(q.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    sA, sB = q.AdamW8State(K * r), q.AdamW8State(N * r)
+
+    def fused():
+        q.lora_grads_adamw8(X, dY, sU, sT, Am, Bm, sA, sB, 1e-4, A_bf16=Ab, B_bf16=Bb)
+
+    def separate():
+        q.lora_grads(X, dY, sU, sT, dA, dB, ws)
+        dAt.copy_(dA.t())
+        q.adamw8_step(Am.view(-1), dAt.view(-1), sA, 1e-4, p_bf16=Ab)
+        q.adamw8_step(Bm.view(-1), dB.view(-1), sB, 1e-4, p_bf16=Bb)
+
+    out = {"workload": "adapter gradients + 8-bit AdamW of A [16 x 4096] and B [4096 x 16], 2048 tokens"}
+    for name, fn in (("fused_us", fused), ("separate_us", separate)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / steps * 1e3
+    return out
+
+
 def bench_mlp_chain(q, torch, steps, warmup):
     """Llama-7B SiLU-gated MLP (gate/up 4096->11008, down 11008->4096), 4096
     tokens, r=16, alpha=32, one training step with gradient checkpointing:
@@ -773,6 +814,7 @@ def main():
         torch.cuda.empty_cache()
         extras["mlp_chain"] = bench_mlp_chain(q, torch, steps=5, warmup=2)
         extras["codec_error"] = codec_error(q, torch)
+        extras["adamw8"] = bench_adamw8(q, torch, steps=20, warmup=3)
     sampler.close()
 
     cpu = None
