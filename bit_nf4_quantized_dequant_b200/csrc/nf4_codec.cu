@@ -7,6 +7,9 @@
 // block, one fp32 second-level scale per group of 256 blocks.
 #include <cuda_fp8.h>
 
+#include <cmath>
+#include <limits>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
@@ -37,27 +40,37 @@ __device__ __forceinline__ float decoded_scale(const uint8_t *scale8, const floa
 }
 
 // code = number of midpoints between adjacent levels that n lies strictly
-// above: the nearest level, ties to the lower one. The midpoints of two float32
-// levels are exact in float64, and so is the comparison.
-template <int BOOK>
-__device__ __forceinline__ uint32_t nearest_level(float n) {
-  constexpr float NF4[16] = QLORA_NF4_LEVELS;
-  constexpr float INT4[16] = QLORA_INT4_LEVELS;
-  const float *L = BOOK == kBookInt4 ? INT4 : NF4;
-  const double x = static_cast<double>(n);
+// above: the nearest level, ties to the lower one. The midpoint m of two
+// float32 levels is exact in float64; for a float32 n, n > m holds exactly
+// when n >= up(m), the smallest float32 above m, so the kernel compares n with
+// the fifteen float32 thresholds up(m_i) (computed on the host in float64).
+struct Thresholds {
+  float t[15];
+};
+
+Thresholds thresholds_for(const float (&L)[16]) {
+  Thresholds th{};
+  for (int i = 0; i < 15; ++i) {
+    const double m = 0.5 * (static_cast<double>(L[i]) + static_cast<double>(L[i + 1]));
+    float f = static_cast<float>(m);
+    if (static_cast<double>(f) <= m) f = std::nextafter(f, std::numeric_limits<float>::infinity());
+    th.t[i] = f;
+  }
+  return th;
+}
+
+__device__ __forceinline__ uint32_t nearest_code(float n, const Thresholds &th) {
   uint32_t code = 0;
 #pragma unroll
-  for (int i = 0; i < 15; ++i) {
-    const double mid = 0.5 * (static_cast<double>(L[i]) + static_cast<double>(L[i + 1]));
-    code += (x > mid) ? 1u : 0u;
-  }
+  for (int i = 0; i < 15; ++i) code += n >= th.t[i] ? 1u : 0u;
   return code;
 }
 
-// One CTA per group of 256 blocks; warp w handles blocks w, w+8, ..., four at
-// a time (four independent 256-byte loads in flight per warp); lane l holds
-// elements 2l and 2l+1 of a block, so the packed byte l of the block is
-// written by lane l.
+// One CTA per group of 256 blocks. A warp load covers two consecutive blocks
+// (lanes 0-15 the first, 16-31 the second, four elements each); warp w takes
+// block pairs w, w + 8, ..., four pairs at a time (four 512-byte loads in
+// flight). Lane l writes the two code bytes of its four elements, so a warp
+// writes the 64 code bytes of its pair in one contiguous store.
 constexpr int kQuantBatch = 4;
 
 template <int BOOK, int DQ>
@@ -65,7 +78,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
                                                            uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scale8,
                                                            float *__restrict__ scale2,
-                                                           int32_t *status) {
+                                                           int32_t *status, const Thresholds th) {
   __shared__ float c1s[kGroup];
   __shared__ float red[8];
   __shared__ float mu_s;
@@ -76,30 +89,39 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
   const int lane = threadIdx.x & 31;
 
   bool bad = false;
-  for (int i0 = warp; i0 < nblk; i0 += 8 * kQuantBatch) {
-    float2 v[kQuantBatch];
+  const int half = lane >> 4, hl = lane & 15;
+  const int npairs = (nblk + 1) / 2;
+  for (int p0 = warp; p0 < npairs; p0 += 8 * kQuantBatch) {
+    float4 v[kQuantBatch];
 #pragma unroll
-    for (int u = 0; u < kQuantBatch; ++u) {   // warp-uniform guard: the block exists or not
-      const int i = i0 + 8 * u;
-      v[u] = i < nblk ? __ldg(reinterpret_cast<const float2 *>(W + (b0 + i) * kBlock) + lane) : make_float2(0.f, 0.f);
+    for (int u = 0; u < kQuantBatch; ++u) {   // warp-uniform pair index; the second block may be missing
+      const int i = 2 * (p0 + 8 * u) + half;
+      v[u] = (p0 + 8 * u < npairs && i < nblk)
+                 ? __ldg(reinterpret_cast<const float4 *>(W + (b0 + i) * kBlock) + hl)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kQuantBatch; ++u) {
-      const int i = i0 + 8 * u;
-      if (i >= nblk) break;
-      const int64_t b = b0 + i;
-      bad |= !isfinite(v[u].x) || !isfinite(v[u].y);
-      float m = fmaxf(fabsf(v[u].x), fabsf(v[u].y));
+      if (p0 + 8 * u >= npairs) break;
+      const int i = 2 * (p0 + 8 * u) + half;
+      bad |= !isfinite(v[u].x) || !isfinite(v[u].y) || !isfinite(v[u].z) || !isfinite(v[u].w);
+      float m = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
 #pragma unroll
-      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      for (int o = 8; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));   // within each half
       constexpr uint32_t kZero = BOOK == kBookInt4 ? 8u : 7u;   // index of the exact zero level
-      uint32_t e0 = kZero, e1 = kZero;
+      uint32_t e0 = kZero, e1 = kZero, e2 = kZero, e3 = kZero;
       if (m > 0.f) {
-        e0 = nearest_level<BOOK>(__fdiv_rn(v[u].x, m));
-        e1 = nearest_level<BOOK>(__fdiv_rn(v[u].y, m));
+        e0 = nearest_code(__fdiv_rn(v[u].x, m), th);
+        e1 = nearest_code(__fdiv_rn(v[u].y, m), th);
+        e2 = nearest_code(__fdiv_rn(v[u].z, m), th);
+        e3 = nearest_code(__fdiv_rn(v[u].w, m), th);
       }
-      codes[b * (kBlock / 2) + lane] = static_cast<uint8_t>((e0 << 4) | e1);
-      if (lane == 0) c1s[i] = m;
+      if (i < nblk) {
+        // bytes 2hl, 2hl+1 of the block: (e0 << 4 | e1), (e2 << 4 | e3)
+        const uint16_t two = static_cast<uint16_t>(((e0 << 4) | e1) | (((e2 << 4) | e3) << 8));
+        reinterpret_cast<uint16_t *>(codes + (b0 + i) * (kBlock / 2))[hl] = two;
+        if (hl == 0) c1s[i] = m;
+      }
     }
   }
   if (bad) set_status(status, 5 /* QLORA_ERR_NONFINITE */);
@@ -207,12 +229,20 @@ cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t 
     if (e != cudaSuccess) return e;
   }
   const unsigned grid = static_cast<unsigned>(ng);
+  static const Thresholds th_nf4 = [] {
+    const float L[16] = QLORA_NF4_LEVELS;
+    return thresholds_for(L);
+  }();
+  static const Thresholds th_int4 = [] {
+    const float L[16] = QLORA_INT4_LEVELS;
+    return thresholds_for(L);
+  }();
   if (dq == kDqFp8)
-    nf4_quantize_kernel<kBookNf4, kDqFp8><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+    nf4_quantize_kernel<kBookNf4, kDqFp8><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_nf4);
   else if (book == kBookInt4)
-    nf4_quantize_kernel<kBookInt4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+    nf4_quantize_kernel<kBookInt4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_int4);
   else
-    nf4_quantize_kernel<kBookNf4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status);
+    nf4_quantize_kernel<kBookNf4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_nf4);
   return cudaGetLastError();
 }
 
