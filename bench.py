@@ -821,6 +821,16 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = oracle_sample()
 
+    # The measured peaks hold a burst figure (a GEMM timed alone) and a
+    # sustained one (a GEMM loop held at the board's power cap). The timed
+    # region is the kernel inside a long run of steps: when the clock sampler
+    # saw the power cap active, the sustained figure is the denominator.
+    clocks = sampler.summary()
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if "sw_power_cap" in clocks.get("reasons", []):
+        gemm_peak, gemm_peak_kind = sustained, f"{peak_kind} bf16 sustained (sw_power_cap active in the timed region)"
+    else:
+        gemm_peak, gemm_peak_kind = peak, f"{peak_kind} bf16 burst"
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -840,14 +850,15 @@ def main():
                        "l2": f"inputs rotate over {n_sets} sets of {per_set/1e6:.0f} MB (> L2)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"kernel": "fused_nf4_gemm_kernel (fwd and dX launches)", "bound": "tensor",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_kind": f"{peak_kind} bf16 burst", "traffic": traffic,
+                         "achieved": achieved, "peak": gemm_peak, "unit": "TFLOP/s", "frac": achieved / gemm_peak,
+                         "peak_kind": gemm_peak_kind, "frac_of_burst": achieved / peak,
+                         "frac_of_sustained": achieved / sustained, "traffic": traffic,
                          "launch_ms_fwd": statistics.mean(fwd_ms), "launch_ms_dx": statistics.mean(dx_ms),
                          "share_of_step": fused_total_ms / (ms_step * K_steps)},
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": LAUNCHES_PER_STEP * K_steps,
-            "clocks": sampler.summary(),
+            "clocks": clocks,
             "cpu_baseline": cpu,
         }
         line.update(extras)
