@@ -122,7 +122,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # distributed plumbing (replicas only: the only collective is the timing max)
 # ---------------------------------------------------------------------------
-def init_dist():
+def init_dist(backend: str = "nccl"):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the
+    launcher). The replicas exchange nothing but the timing maximum; "gloo"
+    runs the same plumbing on CPU processes."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -130,9 +133,12 @@ def init_dist():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return rank, world, local
 
 
@@ -147,9 +153,16 @@ def max_over_ranks(x: float, world: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(world: int, flops_per_step: float, steps: int, ms_total_max: float) -> float:
+    """Whole-job TFLOP/s of N replicas (weak scaling): every rank runs the same
+    steps, the job takes the slowest rank's time."""
+    return world * flops_per_step * steps / (ms_total_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -742,7 +755,7 @@ def main():
     ms_total = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = ms_total / K_steps
     flops = step_flops(M, N, K, r)
-    value = world * flops * K_steps / (ms_total * 1e-3) / 1e12
+    value = replica_value(world, flops, K_steps, ms_total)
 
     fwd_ms = [ev[0].elapsed_time(ev[1]) for ev in evs]
     dx_ms = [ev[2].elapsed_time(ev[3]) for ev in evs]
