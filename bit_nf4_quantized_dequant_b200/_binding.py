@@ -22,7 +22,7 @@ __all__ = [
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "adamw8_step", "AdamW8State", "set_gemm_schedule", "gemm_schedule",
     "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR", "dqfp8_sizes", "dqfp8_quantize", "dqfp8_dequantize",
-    "lora_grads_adamw8",
+    "lora_grads_adamw8", "selftest_bounded_wait",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +44,7 @@ SYMBOLS = [
     "qlora_nf4_merge", "qlora_codec_levels", "qlora_codec_quantize", "qlora_codec_dequantize",
     "qlora_adamw8_step", "qlora_set_gemm_schedule",
     "qlora_dqfp8_sizes", "qlora_dqfp8_quantize", "qlora_dqfp8_dequantize",
-    "qlora_lora_grads_adamw8",
+    "qlora_lora_grads_adamw8", "qlora_selftest_bounded_wait",
 ]
 
 
@@ -130,6 +130,8 @@ def library():
                                             ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                             ctypes.c_float, _P]
     lib.qlora_lora_grads_adamw8.restype = st
+    lib.qlora_selftest_bounded_wait.argtypes = [_P, _P]
+    lib.qlora_selftest_bounded_wait.restype = st
     lib.qlora_codec_levels.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_codec_levels.restype = st
     lib.qlora_codec_quantize.argtypes = [_P, ctypes.POINTER(_NF4), ctypes.c_int32, _P, _P]
@@ -556,3 +558,9 @@ def lora_grads_adamw8(X, dY, sU, sT, A_master, B_master, A_state: AdamW8State, B
     _check(library().qlora_lora_grads_adamw8(_ptr(X), _ptr(dY), M, N, K, _ptr(sU), _ptr(sT), r, _ptr(dA), _ptr(dB),
                                              ctypes.byref(a), ctypes.byref(b), A_state.step, lr, beta1, beta2, eps,
                                              weight_decay, _stream(stream)), "qlora_lora_grads_adamw8")
+
+
+def selftest_bounded_wait(status, stream=None) -> None:
+    """Launch one CTA whose bounded wait runs out (qlora_selftest_bounded_wait);
+    after a synchronise, status (int32 CUDA tensor) holds QLORA_ERR_TIMEOUT."""
+    _check(library().qlora_selftest_bounded_wait(_ptr(status), _stream(stream)), "qlora_selftest_bounded_wait")

@@ -489,6 +489,12 @@ qlora_status_t qlora_adamw8_step(float *p, uint16_t *p_bf16, const float *grad, 
                                    weight_decay, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status_t qlora_selftest_bounded_wait(int32_t *dev_status, qlora_stream_t stream) {
+  if (!dev_status) return QLORA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(dev_status) & 3u) return QLORA_ERR_MISALIGNED;
+  return cuda_status(qlora::launch_bounded_wait_selftest(dev_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qlora_status_t qlora_set_gemm_schedule(int32_t schedule) {
   if (schedule < QLORA_SCHEDULE_AUTO || schedule > QLORA_SCHEDULE_PAIR) return QLORA_ERR_INVALID_ARG;
   qlora::set_gemm_schedule(schedule);

@@ -97,6 +97,9 @@ size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
 
 int device_sm_count();
 
+// One CTA whose bounded mbarrier wait runs out (failure-path self-test).
+cudaError_t launch_bounded_wait_selftest(int32_t *status, cudaStream_t st);
+
 // Fused-GEMM tile schedule (qlora_schedule_t values), process-wide.
 void set_gemm_schedule(int schedule);
 int gemm_schedule();

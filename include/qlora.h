@@ -401,6 +401,16 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const uint16_t *X,
 typedef enum { QLORA_SCHEDULE_AUTO = 0, QLORA_SCHEDULE_SINGLE = 1, QLORA_SCHEDULE_PAIR = 2 } qlora_schedule_t;
 qlora_status_t qlora_set_gemm_schedule(int32_t schedule);
 
+/* Failure-path self-test. Every wait inside the kernels of this library is
+ * bounded: after about one second without progress the waiting thread stops,
+ * the kernel writes QLORA_ERR_TIMEOUT to the device status word and returns,
+ * and the CUDA context stays usable. This call launches one CTA whose wait can
+ * never complete (an mbarrier nothing arrives on), so that the path can be
+ * exercised: after the stream is synchronised, *dev_status (device int32,
+ * 4-byte aligned) holds QLORA_ERR_TIMEOUT. It takes about one second of GPU
+ * time. Errors: INVALID_ARG, MISALIGNED, CUDA. */
+qlora_status_t qlora_selftest_bounded_wait(int32_t *dev_status, qlora_stream_t stream);
+
 /* A static, human-readable name for a status code (host). */
 const char *qlora_status_string(qlora_status_t status);
 

@@ -225,3 +225,24 @@ def test_few_token_forward(lib, N, K, M, r):
     Yr, U = olin.linear_fwd(h["Wd"], h["X"], h["A"], h["B"], s)
     assert_close_fp(bf16_dev_to_f64(sU), s * U, "sU")
     assert_close_fp(bf16_dev_to_f64(Y), Yr, "Y")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(lib):
+    """A kernel wait that can never complete (qlora_selftest_bounded_wait)
+    gives up after the library's limit, writes QLORA_ERR_TIMEOUT to the
+    device status and returns; the same context then runs a linear forward
+    that matches the oracle."""
+    import time
+    import torch
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    lib.selftest_bounded_wait(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 6                      # QLORA_ERR_TIMEOUT
+    assert time.time() - t0 < 30
+    N, K, M, r, s = 256, 512, 40, 16, 2.0
+    h, d = _setup(lib, N, K, M, r, index=11)
+    Y, sU = lib.linear_fwd(d["q"], d["X"], d["A"], d["B"], s)
+    torch.cuda.synchronize()
+    Yr, _ = olin.linear_fwd(h["Wd"], h["X"], h["A"], h["B"], s)
+    assert_close_fp(bf16_dev_to_f64(Y), Yr, "Y after the timeout")
