@@ -15,7 +15,7 @@ The library's main format reads it as unsigned linear absmax codes (nf4.py).
 This module is the comparison format the cited paper describes: the block
 constants of a group are centred on their mean (they are all positive, so
 centring lets a symmetric format use both signs) and stored as 8-bit floats.
-Readings (each listed in the design doc):
+Readings:
   * 8-bit float = E4M3 (4 exponent bits, bias 7, 3 mantissa bits, no
     infinities, largest finite 448); encoding rounds to nearest, ties to an
     even mantissa, and saturates to +-448.

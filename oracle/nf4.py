@@ -16,7 +16,7 @@ Sources (page title, section):
     double quantisation": blockwise quantisation stores one absmax constant
     per block; NF4 levels sit at normal quantiles; 0.5 byte per parameter.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * codebook: 8 positive and 7 negative quantiles plus an exact zero, from the
     construction of the paper the multigrid.ai page cites (arXiv 2305.14314),
     restated here as mathematics; offset NF4_OFFSET (parity unpinned: the
