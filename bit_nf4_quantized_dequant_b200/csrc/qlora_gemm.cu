@@ -21,8 +21,10 @@
 // Three rings decouple the producers from the consumers: packed codes (TMA ->
 // dequantisers, deep, so codes are waiting when a dequantiser gets to them),
 // activations (TMA -> MMA) and dequantised bf16 tiles (dequantisers -> MMA).
-// Two groups of four warps dequantise alternate K-steps, one thread per
-// 64-weight block.
+// Three groups of four warps dequantise every third K-step each, one thread
+// per 64-weight block: a group needs about three MMA K-steps' time for one
+// tile, so with two groups the MMA waited for them (three groups: the DX
+// launch of the 2048-token attention projection 69 -> 65 us, bit-identical).
 //
 // Two variants share this source. Single CTA: UMMA M = 128, one CTA per tile;
 // a K-step of a 256-token tile needs 512 tensor cycles but the dequantisation
@@ -45,10 +47,11 @@
 // (tile, k-step) units are split evenly over all SMs, and tiles cut between
 // CTAs are finished through fp32 partials in the workspace (see GemmParams).
 //
-// Warp roles (512 threads): 0 codes producer, 1 MMA issuer and TMEM owner,
-// 2 activation producer, 3 LoRA-slice producer, 4-7 epilogue (TMEM lane
-// quadrant = warp % 4; results leave through shared memory and TMA stores),
-// 8-11 and 12-15 the two dequantiser groups. Persistent CTAs walk the tile
+// Warp roles (640 threads, 96 registers each; stream-K: 512): 0 codes
+// producer, 1 MMA issuer and TMEM owner, 2 activation producer, 3 LoRA-slice
+// producer, 4-7 epilogue (TMEM lane quadrant = warp % 4; results leave through
+// shared memory and TMA stores), 8-11, 12-15 (and 16-19) the dequantiser
+// groups. Persistent CTAs walk the tile
 // list; the single-CTA TMEM accumulator is double-buffered so the epilogue of
 // one tile overlaps the main loop of the next (a pair's two accumulators take
 // all 512 columns: its next tile's MMAs wait for the epilogue, while its
@@ -60,7 +63,11 @@
 namespace qlora {
 namespace {
 
-constexpr int kThreads = 512;
+// Dequantiser groups of four warps: three for whole tiles; two for stream-K
+// (short token tiles, where the third group's registers cost more than it
+// adds), so the block is 640 or 512 threads.
+__host__ __device__ constexpr int dq_groups(bool streamk) { return streamk ? 2 : 3; }
+__host__ __device__ constexpr int kernel_threads(bool streamk) { return 256 + 128 * dq_groups(streamk); }
 constexpr int kTileRows = 128;                                // weight rows per CTA
 constexpr int kKStage = 64;                                   // K per step (one NF4 block)
 constexpr uint32_t kATileBytes = kTileRows * kKStage * 2;     // 16 KiB
@@ -196,7 +203,7 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int slots, uint32_t i
 // One instantiation per (pair, mode, stream-K) so that each launch carries only
 // the code of its own epilogue: the instruction cache is shared by all roles.
 template <bool kPair, int kMode, bool kStreamK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kernel_threads(kStreamK), 1)
     fused_nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                           const __grid_constant__ CUtensorMap tm_codes,
                           const __grid_constant__ CUtensorMap tm_lora_w,
@@ -730,8 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (et == 0) bulk_wait_group<0>();
   } else {
-    // ---------------- dequantisers: two groups on alternate K-steps ----------------
-    const int g = (threadIdx.x - 256) >> 7;     // group 0 or 1
+    // ---------------- dequantisers: kDqGroups groups, each on every kDqGroups-th K-step ----------------
+    constexpr int kDqGroups = dq_groups(kStreamK);
+    const int g = (threadIdx.x - 256) >> 7;     // group 0 .. kDqGroups - 1
     const int i = (threadIdx.x - 256) & 127;    // block slot inside the step
     // FWD: slot = weight row n (0..127), one block per row per step.
     // DX:  slot = (column block kb in 0..1) * 64 + weight row n (0..63).
@@ -761,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         d = __ldg(p.scale2 + (b >> 8));
       }
     };
-    // Scale loads run three of this group's steps (six steps) ahead; the loop
+    // Scale loads run three of this group's steps ahead; the loop
     // is unrolled by three so each prefetched value stays in its own register
     // until it is used.
     uint32_t qv[3];
@@ -771,15 +779,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     pf.advance(g, p.nk, walk);
 #pragma unroll
     for (int u = 0; u < 3; ++u) {
-      scale_at(pf, 2 * u + g, qv[u], dv[u]);
-      pf.advance(2, p.nk, walk);
+      scale_at(pf, kDqGroups * u + g, qv[u], dv[u]);
+      pf.advance(kDqGroups, p.nk, walk);
     }
-    RingPos cr{g, 0}, ar{g, 0};    // rings of depth >= 2: step g sits in slot g of phase 0
+    RingPos cr{g, 0}, ar{g, 0};    // rings of depth >= kDqGroups: step g sits in slot g of phase 0
     bool ok = true;
     for (int j0 = 0; ok; j0 += 3) {
 #pragma unroll
       for (int u = 0; u < 3; ++u) {
-        const int it = 2 * (j0 + u) + g;
+        const int it = kDqGroups * (j0 + u) + g;
         if (it >= total_steps) { ok = false; break; }
         const int cs = cr.slot, as = ar.slot;
         if (!mbar_wait(&sm.cf[cs], cr.phase, abort_flag, p.status) ||
@@ -806,10 +814,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.af[as]);   // CTA scope; the odd CTA's tiles are forwarded
-        scale_at(pf, it + 6, qv[u], dv[u]);
-        pf.advance(2, p.nk, walk);
-        cr.advance(2, p.sc);
-        ar.advance(2, p.sa);
+        scale_at(pf, it + 3 * kDqGroups, qv[u], dv[u]);
+        pf.advance(kDqGroups, p.nk, walk);
+        cr.advance(kDqGroups, p.sc);
+        ar.advance(kDqGroups, p.sa);
       }
     }
   }
@@ -861,7 +869,7 @@ void pick_rings(int bt_cta, int r_pad, bool pair, int &sx, int &sa, int &sc) {
       if (smem_bytes(bt_cta, r_pad, sx, sa, sc) <= budget) return;
     }
   }
-  const int fallback[][3] = {{3, 3, 4}, {3, 2, 4}, {2, 2, 4}, {2, 2, 3}};
+  const int fallback[][3] = {{3, 3, 4}, {2, 3, 4}, {2, 3, 3}};   // dequantised-tile and code rings >= 3 groups
   for (const auto &f : fallback) {
     sx = f[0];
     sa = f[1];
@@ -989,7 +997,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
     auto go = [&](auto kernel) -> cudaError_t {
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return e;
-      kernel<<<grid, kThreads, smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux, p);
+      kernel<<<grid, kernel_threads(p.streamk != 0), smem, st>>>(tm_act, tm_codes, tm_lw, tm_la, tm_out, tm_aux, p);
       return cudaGetLastError();
     };
     switch (a.mode * 2 + p.streamk) {
@@ -1010,7 +1018,7 @@ cudaError_t launch_fused_gemm(const GemmArgs &a, cudaStream_t st) {
   const int pairs = ntiles < sms / 2 ? ntiles : sms / 2;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kernel_threads(false));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
