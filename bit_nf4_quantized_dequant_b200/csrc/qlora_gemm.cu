@@ -38,9 +38,9 @@
 // and dequantisers signal the even CTA's barriers, and the even CTA's MMA
 // completions are multicast to both; the odd CTA's dequantised tiles reach
 // the even CTA through one forwarding thread (a single cluster-scope release
-// per K-step instead of one per dequantiser warp). On B200 the pair measured
-// no faster than single-CTA tiles (the K-step time grows with its doubled MMA
-// work), so it runs only when the caller selects it (qlora_set_gemm_schedule).
+// per K-step instead of one per dequantiser warp). The launcher takes the pair
+// for large token counts (see use_pair); qlora_set_gemm_schedule can force
+// either variant.
 //
 // Scheduling: persistent CTAs (or pairs) take whole tiles (tile = blockIdx + i * gridDim).
 // With a workspace and token tiles of at most 64, stream-K instead: the
@@ -896,13 +896,28 @@ int token_tile(int64_t M) {
 
 constexpr int kPairTokens = 512;   // token tile of a CTA pair (two N = 256 MMAs)
 
-// The CTA pair runs the linear forward and dX only. On B200 it measured no
-// faster than single-CTA tiles at the shapes of the 7B / 8B linears (the
-// kernel's K-step time grew with the pair's doubled MMA work instead of
-// staying at the dequantisation-bound single-CTA time), so the automatic
-// schedule keeps single CTAs and the pair runs when it is asked for.
+// The CTA pair runs the linear forward and dX only. Each dequantised weight
+// feeds a 512-token tile instead of 256, and each CTA reads half as many
+// activation bytes per flop, so it spends less energy per flop: in short
+// bursts of launches it is a few percent slower than single CTAs, but once
+// the board sits at its power cap (long runs; on the 2048-token attention
+// projection after a few hundred steps) it is faster (step 157 us against
+// 163-167 us). The automatic schedule takes it when its tiles fill the SM
+// pairs about as well as single-CTA tiles fill the SMs.
 bool use_pair(const GemmArgs &a) {
-  return gemm_schedule() == 2 && a.mode <= 1 && a.M > 0;
+  const int sched = gemm_schedule();
+  if (a.mode > 1 || sched == 1) return false;
+  if (sched == 2) return a.M > 0;
+  if (a.M < 2 * kPairTokens) return false;
+  const int64_t rows = a.mode == 1 ? a.K : a.N;
+  const int64_t sms = device_sm_count();
+  const int bt = token_tile(a.M);
+  const int64_t t_single = ((rows + kTileRows - 1) / kTileRows) * ((a.M + bt - 1) / bt);
+  const int64_t t_pair = ((rows + 2 * kTileRows - 1) / (2 * kTileRows)) * ((a.M + kPairTokens - 1) / kPairTokens);
+  const double eff_single = static_cast<double>(t_single) / static_cast<double>(((t_single + sms - 1) / sms) * sms);
+  const int64_t pairs = sms / 2;
+  const double eff_pair = static_cast<double>(t_pair) / static_cast<double>(((t_pair + pairs - 1) / pairs) * pairs);
+  return eff_pair >= 0.95 * eff_single;
 }
 
 std::atomic<int> g_schedule{0};

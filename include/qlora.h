@@ -388,7 +388,12 @@ qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const uint16_t *X,
  * Tile schedule of the fused GEMM (qlora_fused_fwd, qlora_fused_dx and the
  * composite calls that run them). Every schedule computes the same result up to
  * fp32 summation order; this is a tuning and testing control.
- *   QLORA_SCHEDULE_AUTO   the library's choice (default): single-CTA tiles of
+ *   QLORA_SCHEDULE_AUTO   the library's choice (default): CTA pairs for the
+ *                         linear forward and dX at 1024 tokens or more when
+ *                         their tiles fill the SM pairs about as well as
+ *                         single-CTA tiles fill the SMs (fewer dequantisations
+ *                         and activation reads per flop: faster once the board
+ *                         is at its power cap); otherwise single-CTA tiles of
  *                         128 weight rows, stream-K for short token tiles
  *   QLORA_SCHEDULE_SINGLE single-CTA tiles only
  *   QLORA_SCHEDULE_PAIR   CTA pairs (cta_group::2, 256 weight rows x 512 tokens

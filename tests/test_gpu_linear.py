@@ -139,10 +139,11 @@ SCHEDULE_CASES = [
 
 @pytest.mark.parametrize("N,K,M,r", SCHEDULE_CASES)
 def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
-    """qlora_fused_fwd / qlora_fused_dx without a workspace (whole tiles per
-    CTA), with one (stream-K, partial tiles summed through the workspace) and
-    on CTA pairs (cta_group::2, selected with qlora_set_gemm_schedule) all
-    match the oracle; they differ only in fp32 summation order."""
+    """qlora_fused_fwd / qlora_fused_dx with the automatic schedule, forced to
+    single-CTA whole tiles, with a workspace (stream-K for short token tiles,
+    partial tiles summed through the workspace) and forced to CTA pairs
+    (cta_group::2) all match the oracle; they differ only in fp32 summation
+    order."""
     import torch
     s = 2.0
     h, d = _setup(lib, N, K, M, r, index=5)
@@ -156,8 +157,8 @@ def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
     gws = torch.full((lib.fused_workspace(M),), 0xAB, dtype=torch.uint8, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = {}
-    for name, ws, schedule in (("whole", None, lib.SCHEDULE_AUTO), ("streamk", gws, lib.SCHEDULE_AUTO),
-                               ("pair", None, lib.SCHEDULE_PAIR)):
+    for name, ws, schedule in (("auto", None, lib.SCHEDULE_AUTO), ("single", None, lib.SCHEDULE_SINGLE),
+                               ("streamk", gws, lib.SCHEDULE_AUTO), ("pair", None, lib.SCHEDULE_PAIR)):
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         dX = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda")
         with lib.gemm_schedule(schedule):
