@@ -373,34 +373,59 @@ def bench_merge(q, torch, mats, steps, warmup):
             "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats)}
 
 
-def bench_decode(q, torch, mats, steps, warmup):
-    from bit_nf4_quantized_dequant_b200 import inputs
+def bench_decode(q, torch, mats, steps, warmup, concurrent=True):
+    """Forward of every linear of the 8B set at 8 tokens through the composite
+    qlora_linear_fwd (one launch per matrix), captured once in a CUDA graph.
+    With `concurrent`, the linears a decoder layer can issue together because
+    they read the same input (q, k, v; gate, up) run on forked streams, and o
+    and down follow them, as in a layer; otherwise every launch is serial."""
     M, r = 8, 16
     s = 2.0
     g = torch.Generator(device="cuda")
     g.manual_seed(77)
-    per_shape = {}
-    lora = []
+    xs, outs, lora = {}, {}, []
     moved = 0
     for lin, m in mats:
-        key = (lin.N, lin.K)
-        if key not in per_shape:
-            X = (torch.randn((M, lin.K), generator=g, device="cuda")).to(torch.bfloat16)
-            per_shape[key] = dict(X=X, Y=torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda"),
+        if lin.K not in xs:
+            xs[lin.K] = (torch.randn((M, lin.K), generator=g, device="cuda")).to(torch.bfloat16)
+        if lin.name not in outs:
+            outs[lin.name] = dict(Y=torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda"),
                                   sU=torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
                                   ws=torch.empty(q.linear_workspace(M, lin.N, lin.K, r), dtype=torch.uint8,
-                                                 device="cuda"),
-                                  gws=torch.empty(q.fused_workspace(M), dtype=torch.uint8, device="cuda"))
+                                                 device="cuda"))
         A = (torch.randn((r, lin.K), generator=g, device="cuda") / r).to(torch.bfloat16)
         B = (torch.randn((lin.N, r), generator=g, device="cuda") * 0.01).to(torch.bfloat16)
         lora.append((A, B))
         moved += sum(q.nf4_sizes(lin.N, lin.K)) + 2 * r * (lin.N + lin.K) + 2 * M * (lin.N + lin.K)
+    together = {"q": "qkv", "k": "qkv", "v": "qkv", "gate": "gu", "up": "gu"}
+    side = [torch.cuda.Stream() for _ in range(2)]
+
+    def launch(i):
+        (lin, m), (A, B) = mats[i], lora[i]
+        o = outs[lin.name]
+        q.linear_fwd(m, xs[lin.K], A, B, s, Y=o["Y"], sU=o["sU"], ws=o["ws"])
 
     def one_pass():
         # the composite forward: at 8 tokens one launch per matrix forms sU and Y
-        for (lin, m), (A, B) in zip(mats, lora):
-            d = per_shape[(lin.N, lin.K)]
-            q.linear_fwd(m, d["X"], A, B, s, Y=d["Y"], sU=d["sU"], ws=d["ws"])
+        i = 0
+        while i < len(mats):
+            grp = together.get(mats[i][0].name) if concurrent else None
+            j = i + 1
+            while grp is not None and j < len(mats) and together.get(mats[j][0].name) == grp:
+                j += 1
+            if j - i == 1:
+                launch(i)
+            else:
+                main = torch.cuda.current_stream()
+                for k in range(i + 1, j):
+                    side[k - i - 1].wait_stream(main)
+                launch(i)
+                for k in range(i + 1, j):
+                    with torch.cuda.stream(side[k - i - 1]):
+                        launch(k)
+                for k in range(i + 1, j):
+                    main.wait_stream(side[k - i - 1])
+            i = j
 
     for _ in range(warmup):
         one_pass()
@@ -428,7 +453,8 @@ def bench_decode(q, torch, mats, steps, warmup):
     alu_peak = 64 * torch.cuda.get_device_properties(0).multi_processor_count * ALU_CLOCK_HZ
     return {"workload": "set_8b forward at 8 tokens: 224 matrices, r=16", "GB/s": moved / ms / 1e6,
             "bytes_per_pass": moved, "ms_per_pass": ms, "launches_per_pass": len(mats),
-            "launch": "CUDA graph of the pass",
+            "launch": "CUDA graph of the pass" + ("; q, k, v and gate, up of a layer on forked streams"
+                                                   if concurrent else ", serial"),
             "roofline": {"kernel": "nf4_gemv_fwd_kernel", "bound": "alu", "achieved": alu_ops / (ms * 1e-3) / 1e12,
                          "peak": alu_peak / 1e12, "unit": "T ALU lane-ops/s", "frac": alu_ops / (ms * 1e-3) / alu_peak,
                          "ops_per_weight": 21 / 8 + 8 / 64,
