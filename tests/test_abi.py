@@ -126,3 +126,42 @@ def test_gemm_schedule_control(lib):
     with lib.gemm_schedule(lib.SCHEDULE_PAIR):
         pass
     assert so.qlora_set_gemm_schedule(lib.SCHEDULE_AUTO) == 0
+
+
+def test_argument_errors_of_the_next_scope_calls(lib):
+    """The comparison second level, the fused gradient + AdamW launch and the
+    failure-path self-test refuse bad arguments before any launch."""
+    so = lib.library()
+    SZ, P = ctypes.c_size_t, ctypes.c_void_p
+    a, b, c = SZ(), SZ(), SZ()
+    assert so.qlora_dqfp8_sizes(64, 256, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)) == 0
+    assert (a.value, b.value, c.value) == (64 * 128, 256, 8)        # (d, mu) per group: 8 bytes
+    n1, n2, n3 = SZ(), SZ(), SZ()
+    so.qlora_nf4_sizes(4096, 4096, ctypes.byref(n1), ctypes.byref(n2), ctypes.byref(n3))
+    so.qlora_dqfp8_sizes(4096, 4096, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    assert (a.value, b.value, c.value) == (n1.value, n2.value, 2 * n3.value)
+    q = _nf4(16, 64)
+    assert so.qlora_dqfp8_quantize(None, ctypes.byref(q), None, None) == 1
+    q4 = _nf4(16, 64, s2=0x30004)                                    # 4-byte but not 8-byte aligned
+    assert so.qlora_dqfp8_quantize(P(0x40000), ctypes.byref(q4), None, None) == 3
+    assert so.qlora_dqfp8_dequantize(ctypes.byref(q4), P(0x40000), None) == 3
+    assert so.qlora_dqfp8_dequantize(ctypes.byref(q), None, None) == 1
+    # fused gradients + AdamW
+    from bit_nf4_quantized_dequant_b200._binding import _Adam8
+    st = _Adam8(0x100000, 0, 0x110000, 0x120000, 0x130000, 0x140000)
+    X, dY, sU, sT = P(0x50000), P(0x60000), P(0x70000), P(0x80000)
+    g = so.qlora_lora_grads_adamw8
+    args = lambda **k: dict(dict(r=16, A=ctypes.byref(st), B=ctypes.byref(st), step=1, lr=1e-4, b1=0.9, b2=0.999,
+                                 eps=1e-8), **k)
+    call = lambda d: g(X, dY, 64, 256, 128, sU, sT, d["r"], None, None, d["A"], d["B"], d["step"], d["lr"],
+                       d["b1"], d["b2"], d["eps"], 0.0, None)
+    assert call(args(A=None)) == 1
+    assert call(args(step=0)) == 1
+    assert call(args(b1=1.0)) == 1
+    assert call(args(eps=0.0)) == 1
+    assert call(args(r=12)) == 2
+    bad = _Adam8(0x100000, 0, 0, 0x120000, 0x130000, 0x140000)       # missing m_q
+    assert call(args(B=ctypes.byref(bad))) == 1
+    # self-test
+    assert so.qlora_selftest_bounded_wait(None, None) == 1
+    assert so.qlora_selftest_bounded_wait(P(0x50002), None) == 3
