@@ -148,8 +148,12 @@ qlora_status_t qlora_dqfp8_quantize(const float *W, const qlora_nf4_t *q, int32_
 qlora_status_t qlora_dqfp8_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora_stream_t stream);
 
 /* Workspace bytes that qlora_linear_fwd and qlora_linear_bwd need for M
- * tokens through an [N, K] layer of rank r (host). The same workspace may be
- * reused by consecutive calls on one stream; calls that run concurrently need
+ * tokens through an [N, K] layer of rank r (host). Interface only: no passage
+ * of the pages defines it; it exists because this library never allocates, so
+ * the caller sizes and owns the scratch memory the kernels use. It takes
+ * (M, N, K, r) rather than the weight itself so that a caller can size the
+ * workspace before any weight is quantised. The same workspace may be reused
+ * by consecutive calls on one stream; calls that run concurrently need
  * separate workspaces. Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
 qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r,
                                       size_t *bytes);
@@ -416,7 +420,9 @@ qlora_status_t qlora_set_gemm_schedule(int32_t schedule);
  * time. Errors: INVALID_ARG, MISALIGNED, CUDA. */
 qlora_status_t qlora_selftest_bounded_wait(int32_t *dev_status, qlora_stream_t stream);
 
-/* A static, human-readable name for a status code (host). */
+/* A static, human-readable name for a status code (host). Interface only:
+ * no passage of the pages defines it; it turns the codes above into text for
+ * error messages. Never NULL; unknown codes give "QLORA_ERR_UNKNOWN". */
 const char *qlora_status_string(qlora_status_t status);
 
 #ifdef __cplusplus

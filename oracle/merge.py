@@ -32,9 +32,16 @@ def requant_drift(merged_f32: np.ndarray, Wd: np.ndarray, A: np.ndarray, B: np.n
     """Quantise the merged weight to NF4 again and compare its dequantised
     value with the exact merge. Returns (relative Frobenius error of the
     re-quantised merge against the exact merge, the same error divided by the
-    norm of the adapter's contribution s B A)."""
+    norm of the adapter's contribution s B A). A ratio whose denominator is
+    zero (a zero adapter, or a zero merge) is inf when the drift is not zero
+    and NaN when it is."""
     N, K = merged_f32.shape
     back = nf4.dequantize(*nf4.quantize(merged_f32), N, K)
     exact = merge(Wd, A, B, s)
     err = np.linalg.norm(back - exact)
-    return err / np.linalg.norm(exact), err / np.linalg.norm(exact - np.asarray(Wd, dtype=np.float64))
+    ref = np.linalg.norm(exact)
+    delta = np.linalg.norm(exact - np.asarray(Wd, dtype=np.float64))
+    # a zero merge or a zero adapter leaves a ratio undefined: inf when there
+    # is drift to relate to nothing, NaN when there is none
+    ratio = lambda den: err / den if den > 0 else (np.inf if err > 0 else np.nan)
+    return ratio(ref), ratio(delta)

@@ -248,3 +248,120 @@ def test_row_and_column_restrictions_equal_the_whole(N, K):
     np.testing.assert_array_equal(pr, packed.reshape(N, K // 2)[rows])
     np.testing.assert_array_equal(s8r, s8.reshape(N, K // 64)[rows])
     np.testing.assert_array_equal(s2r, s2)
+
+
+def _midpoint_scales(levels: np.ndarray, per_level: int, rng) -> list:
+    """Float32 scales s for which RN32(level * s) is exactly halfway between
+    two bf16 values (low 16 bits 0x8000) while the exact product is not: the
+    products where rounding to float32 first and then to bf16 differs from
+    one rounding of the exact product whenever the exact product lies on the
+    side of the odd bf16 neighbour. Levels 0 and +-1 have exact products and
+    are skipped."""
+    out = []
+    for i, L in enumerate(levels.astype(np.float64)):
+        if L == 0.0 or abs(L) == 1.0:
+            continue
+        found = 0
+        for _ in range(50 * per_level):
+            if found == per_level:
+                break
+            t_bits = (int(rng.integers(0x3C000000, 0x3F000000)) & 0xFFFF0000) | 0x8000
+            t = float(np.array([t_bits], np.uint32).view(np.float32)[0]) * (1.0 if L > 0 else -1.0)
+            s0 = np.float32(t / L)
+            for k in range(-3, 4):
+                s = s0
+                for _ in range(abs(k)):
+                    s = np.nextafter(s, np.float32(np.inf) if k > 0 else np.float32(-np.inf))
+                exact = Fraction(float(L)) * Fraction(float(s))
+                if float(np.float32(float(exact))) == t and exact != Fraction(t):
+                    out.append((i, np.float32(s)))
+                    found += 1
+                    break
+    return out
+
+
+def _bf16_single_rounding(x: Fraction) -> int:
+    """bf16 bits of one round-to-nearest-even rounding of an exact value
+    (finite, within the normal float32 range or zero)."""
+    if x == 0:
+        return 0
+    sign = 0x8000 if x < 0 else 0
+    m = abs(x)
+    b = int(np.array([np.float32(float(m))], np.float32).view(np.uint32)[0]) & 0xFFFF0000
+    cands = []
+    for hi in (b - 0x10000, b, b + 0x10000):
+        if hi < 0:
+            continue
+        v = Fraction(float(np.array([hi], np.uint32).view(np.float32)[0]))
+        cands.append((abs(v - m), (hi >> 16) & 1, hi >> 16))
+    cands.sort()
+    if cands[0][0] == cands[1][0]:                # exact tie: the even one
+        return (min(cands[:2], key=lambda c: c[1])[2] & 0x7FFF) | sign
+    return (cands[0][2] & 0x7FFF) | sign
+
+
+def _rounding_case():
+    """Blocks that each hold all 16 codes four times, with block scales
+    s = RN32(q8 * d) that vary per block: 512 groups of random scales, then one
+    group per crafted midpoint scale (its first block has q8 = 1, so s = d).
+    Returns the codec inputs, torch's float32-then-bf16 bits and the crafted
+    (block, level) pairs with their exact single-rounding bits."""
+    rng = np.random.Generator(np.random.PCG64(11))
+    levels = nf4.nf4_levels()
+    crafted = _midpoint_scales(levels, 12, rng)
+    n_groups = 512 + len(crafted)
+    codes = np.tile(np.arange(16, dtype=np.uint8), 4)
+    nb = n_groups * 256
+    q8 = rng.integers(1, 256, nb).astype(np.uint8)
+    d = (rng.uniform(0.5, 2.0, n_groups) * 10.0 ** rng.integers(-6, 1, n_groups)).astype(np.float32)
+    for g, (_, s) in enumerate(crafted):
+        q8[(512 + g) * 256] = 1
+        d[512 + g] = s
+    packed = nf4.pack_codes(np.tile(codes, nb))
+    s_t = torch.from_numpy(q8.astype(np.float32)) * torch.from_numpy(np.repeat(d, 256))   # float32 products
+    w_t = torch.from_numpy(levels)[torch.from_numpy(codes.astype(np.int64))][None, :] * s_t[:, None]
+    ref = w_t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    single = [((512 + g) * 256, i, _bf16_single_rounding(Fraction(float(levels[i])) * Fraction(float(s))))
+              for g, (i, s) in enumerate(crafted)]
+    return packed, q8, d, nb, ref, single
+
+
+def test_dequant_rounding_matches_float32_then_bf16_in_torch():
+    """The dequantiser's rounding reading, w' = RN_bf16(RN32(level * s)) with
+    s = RN32(q8 * d) ("QLoRA, in depth", "The mechanism in brief": the weight
+    is dequantised to the bf16 compute dtype through the float32 block
+    constant), against torch's own float32 multiplies and bf16 cast: all 16
+    levels times about 1.3e5 float32 scales, plus crafted scales whose float32
+    product sits exactly on a bf16 midpoint while the exact product does not.
+    One rounding of the exact product straight to bf16 (the neighbouring
+    reading) gives other bits on part of the crafted cases."""
+    packed, q8, d, nb, ref, single = _rounding_case()
+    bits = nf4.dequantize_bits(packed, q8, d, nb, 64).reshape(nb, 64)
+    assert np.array_equal(bits, ref)
+    differ = sum(1 for b, i, sb in single if sb != int(bits[b, i]))
+    assert len(single) >= 150 and differ >= len(single) // 4
+
+
+def test_planted_single_rounding_is_caught(monkeypatch):
+    """A dequantiser that rounds the exact product once, straight to bf16,
+    passes every bound and special value but fails the pin above."""
+    def one_rounding(packed, scale8, scale2, rows, cols):
+        levels = nf4.nf4_levels().astype(np.float64)
+        codes = nf4.unpack_codes(packed).reshape(-1, nf4.BLOCK)
+        s = nf4.block_scales(scale8, scale2).astype(np.float64)
+        v = (levels[codes] * s[:, None]).reshape(-1)        # exact in float64
+        a = np.abs(v)
+        ulp = np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7)
+        lo = np.floor(a / ulp)                              # exact: scaling by powers of two
+        frac = a / ulp - lo
+        up = (frac > 0.5) | ((frac == 0.5) & (lo % 2 == 1))
+        r = np.where(a > 0, (lo + up) * ulp, 0.0) * np.sign(v)
+        return nf4.bf16_round_bits(r.astype(np.float32)).reshape(rows, cols)   # r is already on the bf16 grid
+
+    packed, q8, d, nb, ref, single = _rounding_case()
+    # the crafted groups alone keep the planted version fast
+    sel = slice(512 * 256, nb)
+    sub = nf4.pack_codes(nf4.unpack_codes(packed).reshape(nb, 64)[sel].reshape(-1))
+    monkeypatch.setattr(nf4, "dequantize_bits", one_rounding)
+    bits = nf4.dequantize_bits(sub, q8[sel], d[512:], nb - 512 * 256, 64)
+    assert not np.array_equal(bits, ref[sel])

@@ -36,8 +36,9 @@ def test_requant_of_the_base_alone_is_not_exact():
     again), so even a zero adapter drifts by a little: the pages' warning
     about requantising merged weights holds before any adapter is added."""
     Wd, A, B = _case(seed=403)
-    rel, _ = merge.requant_drift(Wd.astype(np.float32), Wd, A, np.full_like(B, 0.0) + 1e-30, 0.0)
+    rel, rel_delta = merge.requant_drift(Wd.astype(np.float32), Wd, A, np.zeros_like(B), 0.0)
     assert 0.0 < rel < 0.05
+    assert rel_delta == np.inf          # drift against an adapter contribution of zero
 
 
 def test_requant_drift_is_positive_with_an_adapter():
