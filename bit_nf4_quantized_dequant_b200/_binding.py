@@ -22,7 +22,8 @@ __all__ = [
     "nf4_merge", "codec_levels", "codec_quantize", "codec_dequantize", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "adamw8_step", "AdamW8State", "set_gemm_schedule", "gemm_schedule",
     "SCHEDULE_AUTO", "SCHEDULE_SINGLE", "SCHEDULE_PAIR", "dqfp8_sizes", "dqfp8_quantize", "dqfp8_dequantize",
-    "lora_grads_adamw8", "selftest_bounded_wait",
+    "lora_grads_adamw8", "selftest_bounded_wait", "linear_fwd_group", "linear_fwd_group_workspace",
+    "LinearProblem", "FWD_OVERLAP_PREVIOUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -45,6 +46,7 @@ SYMBOLS = [
     "qlora_adamw8_step", "qlora_set_gemm_schedule",
     "qlora_dqfp8_sizes", "qlora_dqfp8_quantize", "qlora_dqfp8_dequantize",
     "qlora_lora_grads_adamw8", "qlora_selftest_bounded_wait",
+    "qlora_linear_fwd_group_workspace", "qlora_linear_fwd_group",
 ]
 
 
@@ -67,6 +69,13 @@ class _NF4(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("scale8", ctypes.c_void_p), ("scale2", ctypes.c_void_p)]
 
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("W", _NF4), ("X", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("r", ctypes.c_int32), ("s", ctypes.c_float), ("Y", ctypes.c_void_p), ("sU_out", ctypes.c_void_p)]
+
+
+FWD_OVERLAP_PREVIOUS = 1
 
 _lib = None
 _P = ctypes.c_void_p
@@ -152,6 +161,12 @@ def library():
     lib.qlora_linear_fwd_noalloc.argtypes = [ctypes.POINTER(_NF4), _P, _I64, _P, _P, ctypes.c_int32,
                                              ctypes.c_float, _P, _P, _P, _P]
     lib.qlora_linear_fwd_noalloc.restype = st
+    lib.qlora_linear_fwd_group_workspace.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _I64,
+                                                     ctypes.POINTER(_SZ)]
+    lib.qlora_linear_fwd_group_workspace.restype = st
+    lib.qlora_linear_fwd_group.argtypes = [ctypes.POINTER(_Problem), ctypes.c_int32, _I64, ctypes.c_int32, _P, _SZ,
+                                           _P, _P]
+    lib.qlora_linear_fwd_group.restype = st
     lib.qlora_status_string.argtypes = [ctypes.c_int]
     lib.qlora_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -283,6 +298,50 @@ def linear_bwd(q: NF4Matrix, X, A, B, s: float, dY, sU=None, dX=None, dA=None, d
                                       _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _ptr(status),
                                       _stream(stream)), "qlora_linear_bwd")
     return dX, dA, dB
+
+
+@dataclass
+class LinearProblem:
+    """One linear of a grouped few-token forward: Y = X W'^T + s (X A^T) B^T."""
+    q: NF4Matrix
+    X: object
+    A: object
+    B: object
+    s: float
+    Y: object
+    sU: object = None
+
+    def c_struct(self) -> _Problem:
+        return _Problem(self.q.c_struct(), self.X.data_ptr(), self.A.data_ptr(), self.B.data_ptr(),
+                        self.A.shape[0], self.s, self.Y.data_ptr(), None if self.sU is None else self.sU.data_ptr())
+
+
+def _problem_array(problems):
+    arr = (_Problem * len(problems))()
+    for i, p in enumerate(problems):
+        arr[i] = p.c_struct()
+    return arr
+
+
+def linear_fwd_group_workspace(problems, M: int) -> int:
+    b = _SZ()
+    _check(library().qlora_linear_fwd_group_workspace(_problem_array(problems), len(problems), M, ctypes.byref(b)),
+           "qlora_linear_fwd_group_workspace")
+    return b.value
+
+
+def linear_fwd_group(problems, ws=None, flags: int = 0, status=None, stream=None, arr=None):
+    """Few-token forward (M <= 16) of several linears in one launch. `arr` may
+    hold a prebuilt ctypes problem array (e.g. for repeated calls)."""
+    import torch
+    M = problems[0].X.shape[0]
+    if arr is None:
+        arr = _problem_array(problems)
+    if ws is None:
+        ws = torch.empty(linear_fwd_group_workspace(problems, M), dtype=torch.uint8, device=problems[0].X.device)
+    _check(library().qlora_linear_fwd_group(arr, len(problems), M, flags, _ptr(ws), ws.numel(), _ptr(status),
+                                            _stream(stream)), "qlora_linear_fwd_group")
+    return [p.Y for p in problems]
 
 
 # ---- the individual steps of the layer ---------------------------------------

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "qlora.h"
 #include "qlora_device.cuh"
@@ -58,6 +59,34 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, ui
   return r == CUDA_SUCCESS;
 }
 
+// Workspace of the few-token forward of one [N, K] linear of rank r that forms
+// sU itself and keeps it in the workspace (the largest case).
+static size_t small_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
+  SmallProblem p{};
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.A = reinterpret_cast<const uint16_t *>(16);   // only "given / not given" matters here
+  return small_m_ws_bytes(&p, 1, M);
+}
+// ... and of the few-token qlora_fused_fwd, which is given sU.
+static size_t small_fused_ws_bytes(int64_t M) {
+  SmallProblem p{};
+  p.N = 16;
+  p.K = 64;
+  p.r = 8;
+  return small_m_ws_bytes(&p, 1, M);
+}
+
+// The optional workspace of qlora_fused_fwd / qlora_fused_dx: the stream-K
+// partials of the GEMM, or for a few tokens the persistent forward's.
+static size_t fused_ws_bytes(int64_t M) {
+  const size_t g = fused_gemm_ws_bytes(M);
+  if (M > kSmallM) return g;
+  const size_t sm = small_fused_ws_bytes(M);
+  return sm > g ? sm : g;
+}
+
 // Workspace layout of the linear calls (offsets in bytes, 256-byte aligned):
 //   [sU scratch: M*r bf16][sT: M*r bf16][fp32 partial sums of the skinny products]
 //   [stream-K workspace of the fused GEMMs]
@@ -78,6 +107,10 @@ static WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r) {
   w.part_floats = f;
   w.gemm = w.part + round_up(f * 4, 256);
   w.gemm_bytes = fused_gemm_ws_bytes(M);
+  if (M <= kSmallM) {   // the few-token forward uses this region instead
+    const size_t sm = small_fwd_ws_bytes(M, N, K, r);
+    w.gemm_bytes = sm > w.gemm_bytes ? sm : w.gemm_bytes;
+  }
   w.total = w.gemm + round_up(w.gemm_bytes, 256);
   return w;
 }
@@ -108,18 +141,61 @@ static qlora_status_t check_linear(const qlora_nf4_t *W, const uint16_t *X, int6
 
 static qlora_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
-// Forward for a few tokens in one launch (sU formed inside); validates like
-// qlora_linear_fwd apart from the workspace, which it does not use.
-qlora_status_t few_token_forward(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
-                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
-                                 qlora_stream_t stream) {
+qlora_status_t linear_fwd_check(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                const uint16_t *B, int32_t r, float s, const uint16_t *Y, const uint16_t *sU_out,
+                                const int32_t *dev_status) {
   qlora_status_t st = check_linear(W, X, M, A, B, r, s);
   if (st != QLORA_OK) return st;
   if (!Y) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(Y) || (sU_out && !aligned16(sU_out))) return QLORA_ERR_MISALIGNED;
-  if (!gemv_fwd_supported(W->rows, W->cols, M)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, X, B, nullptr, A, s,
-                                         sU_out, r, Y, reinterpret_cast<cudaStream_t>(stream)));
+  if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+size_t linear_fwd_scratch_bytes(int64_t M, int64_t N, int64_t K, int32_t r, bool keep_su) {
+  if (M <= kSmallM) {
+    SmallProblem p{};
+    p.N = N;
+    p.K = K;
+    p.r = r;
+    p.A = reinterpret_cast<const uint16_t *>(16);
+    p.sU_out = keep_su ? reinterpret_cast<uint16_t *>(16) : nullptr;
+    return small_m_ws_bytes(&p, 1, M);
+  }
+  size_t b = keep_su ? 0 : round_up(static_cast<size_t>(M) * r * 2, 256);
+  if (M <= 64) b += round_up(fused_gemm_ws_bytes(M), 256);   // the stream-K schedule of short token tiles
+  return b;
+}
+
+// The forward after validation. su_scratch: [M, r] bf16 for sU when sU_out is
+// NULL and M > kSmallM; gemm_ws: the fused GEMM's workspace (M > kSmallM) or
+// the few-token launch's (M <= kSmallM).
+qlora_status_t linear_fwd_run(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                              const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
+                              uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes, int32_t *dev_status,
+                              qlora_stream_t stream) {
+  const int64_t N = W->rows, K = W->cols;
+  if (M <= kSmallM) {
+    SmallProblem p{};
+    p.codes = W->codes;
+    p.scale8 = W->scale8;
+    p.scale2 = W->scale2;
+    p.N = N;
+    p.K = K;
+    p.X = X;
+    p.A = A;
+    p.B = B;
+    p.r = r;
+    p.s = s;
+    p.Y = Y;
+    p.sU_out = sU_out;
+    if (!gemm_ws || gemm_ws_bytes < small_m_ws_bytes(&p, 1, M)) return QLORA_ERR_WORKSPACE;
+    return cuda_status(launch_small_m(&p, 1, M, gemm_ws, false, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+  }
+  uint16_t *sU = sU_out ? sU_out : su_scratch;
+  qlora_status_t st = qlora_lora_xa(X, M, K, A, r, s, sU, nullptr, 0, stream);
+  if (st != QLORA_OK) return st;
+  return qlora_fused_fwd(W, X, M, B, r, sU, Y, gemm_ws, gemm_ws_bytes, dev_status, stream);
 }
 
 }  // namespace qlora
@@ -258,7 +334,7 @@ qlora_status_t qlora_lora_dyb(const uint16_t *dY, int64_t M, int64_t N, const ui
 
 qlora_status_t qlora_fused_workspace(int64_t M, size_t *bytes) {
   if (!bytes || M < 1) return QLORA_ERR_INVALID_ARG;
-  *bytes = fused_gemm_ws_bytes(M);
+  *bytes = fused_ws_bytes(M);
   return QLORA_OK;
 }
 
@@ -269,7 +345,7 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   if (st != QLORA_OK) return st;
   if (!lora_act || !out) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(lora_act) || !aligned16(out) || (ws && !aligned16(ws))) return QLORA_ERR_MISALIGNED;
-  if (ws && ws_bytes < fused_gemm_ws_bytes(M)) return QLORA_ERR_WORKSPACE;
+  if (ws && ws_bytes < fused_ws_bytes(M)) return QLORA_ERR_WORKSPACE;
   if (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return QLORA_ERR_MISALIGNED;
   GemmArgs g{};
   g.mode = mode;
@@ -286,7 +362,22 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   g.out = out;
   g.dev_status = dev_status;
   g.ws = ws;
-  if (mode == 0 && gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens: the weight-streaming kernel
+  if (mode == 0 && M <= kSmallM && ws && W->rows <= INT32_MAX && W->cols <= INT32_MAX) {
+    // a few tokens with a workspace: the persistent weight-streaming launch
+    SmallProblem p{};
+    p.codes = W->codes;
+    p.scale8 = W->scale8;
+    p.scale2 = W->scale2;
+    p.N = W->rows;
+    p.K = W->cols;
+    p.X = act;
+    p.B = lora_w;
+    p.sU_in = lora_act;
+    p.r = r;
+    p.Y = out;
+    return cuda_status(launch_small_m(&p, 1, M, ws, false, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+  }
+  if (mode == 0 && gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens, no workspace: one cluster launch
     return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, act, lora_w,
                                            lora_act, nullptr, 0.f, nullptr, r, out,
                                            reinterpret_cast<cudaStream_t>(stream)));
@@ -354,20 +445,65 @@ qlora_status_t qlora_lora_grads_adamw8(const uint16_t *X, const uint16_t *dY, in
 qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
                                 void *ws, size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
-  qlora_status_t st = check_linear(W, X, M, A, B, r, s);
+  qlora_status_t st = linear_fwd_check(W, X, M, A, B, r, s, Y, sU_out, dev_status);
   if (st != QLORA_OK) return st;
-  if (!Y) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(Y) || (sU_out && !aligned16(sU_out))) return QLORA_ERR_MISALIGNED;
   const int64_t N = W->rows, K = W->cols;
   const WsLayout L = ws_layout(M, N, K, r);
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
-  if (gemv_fwd_supported(N, K, M)) return few_token_forward(W, X, M, A, B, r, s, Y, sU_out, stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws);
-  uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(wsb + L.su);
-  st = qlora_lora_xa(X, M, K, A, r, s, sU, wsb + L.part, L.part_floats * 4, stream);
-  if (st != QLORA_OK) return st;
-  return qlora_fused_fwd(W, X, M, B, r, sU, Y, wsb + L.gemm, L.gemm_bytes, dev_status, stream);
+  return linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, reinterpret_cast<uint16_t *>(wsb + L.su), wsb + L.gemm,
+                        L.gemm_bytes, dev_status, stream);
+}
+
+qlora_status_t qlora_linear_fwd_group_workspace(const qlora_linear_problem_t *problems, int32_t count, int64_t M,
+                                                size_t *bytes) {
+  if (!problems || !bytes || count < 1 || M < 1) return QLORA_ERR_INVALID_ARG;
+  if (M > kSmallM) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  std::vector<SmallProblem> pr(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const qlora_linear_problem_t &q = problems[i];
+    if (q.W.rows <= 0 || q.W.cols <= 0) return QLORA_ERR_INVALID_ARG;
+    if (q.W.cols % kBlock || q.r < 8 || q.r > 64 || q.r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    pr[i].N = q.W.rows;
+    pr[i].K = q.W.cols;
+    pr[i].r = q.r;
+    pr[i].A = q.A;
+    pr[i].sU_out = q.sU_out;
+  }
+  *bytes = small_m_ws_bytes(pr.data(), count, M);
+  return QLORA_OK;
+}
+
+qlora_status_t qlora_linear_fwd_group(const qlora_linear_problem_t *problems, int32_t count, int64_t M, int32_t flags,
+                                      void *ws, size_t ws_bytes, int32_t *dev_status, qlora_stream_t stream) {
+  if (!problems || count < 1 || M < 1) return QLORA_ERR_INVALID_ARG;
+  if (M > kSmallM) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (flags & ~QLORA_FWD_OVERLAP_PREVIOUS) return QLORA_ERR_INVALID_ARG;
+  std::vector<SmallProblem> pr(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    const qlora_linear_problem_t &q = problems[i];
+    qlora_status_t st = linear_fwd_check(&q.W, q.X, M, q.A, q.B, q.r, q.s, q.Y, q.sU_out, dev_status);
+    if (st != QLORA_OK) return st;
+    if (q.W.rows > INT32_MAX || q.W.cols > INT32_MAX) return QLORA_ERR_UNSUPPORTED_SHAPE;
+    SmallProblem &p = pr[i];
+    p.codes = q.W.codes;
+    p.scale8 = q.W.scale8;
+    p.scale2 = q.W.scale2;
+    p.N = q.W.rows;
+    p.K = q.W.cols;
+    p.X = q.X;
+    p.A = q.A;
+    p.B = q.B;
+    p.r = q.r;
+    p.s = q.s;
+    p.Y = q.Y;
+    p.sU_out = q.sU_out;
+  }
+  if (!ws || ws_bytes < small_m_ws_bytes(pr.data(), count, M)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  return cuda_status(launch_small_m(pr.data(), count, M, ws, (flags & QLORA_FWD_OVERLAP_PREVIOUS) != 0, dev_status,
+                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,

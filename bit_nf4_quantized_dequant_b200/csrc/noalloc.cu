@@ -1,14 +1,17 @@
 // Allocation-free variant of the QLoRA linear forward.
 //
-// qlora_linear_fwd needs a caller-provided workspace for the partial sums of
-// s X A^T (and for sU when the caller does not keep it). Some callers have no
+// qlora_linear_fwd needs a caller-provided workspace: for a few tokens the
+// partial sums and flags of its persistent launch and the pieces of s X A^T,
+// for more tokens sU (when the caller does not keep it) and, up to 64 tokens,
+// the fp32 partial tiles of the GEMM's stream-K schedule. Some callers have no
 // way to provide one at the point where they run the layer: a host that hands
 // the library only its inputs and outputs and owns no allocator of its own (a
 // plug-in inside someone else's runtime), a serving process that has given all
 // device memory to a fixed pool up front, or code that must not call
 // cudaMalloc between launches because that call can synchronise the device.
 // For them, qlora_linear_fwd_noalloc takes its scratch from one fixed array
-// compiled into this library instead of from the caller.
+// compiled into this library instead of from the caller, and otherwise runs
+// exactly the launches qlora_linear_fwd runs, so the results are the same bits.
 //
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds kNoAllocScratchBytes of it until the process exits. Host code
@@ -29,7 +32,8 @@ constexpr int kMaxDevices = 64;
 }  // namespace
 
 // The shared scratch. Nothing in it has to start at zero: each call writes
-// every byte it later reads (the partial sums and, if used, sU).
+// every byte it later reads, and the counters of the few-token launch carry a
+// per-launch value that makes stale contents count as zero.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -60,20 +64,21 @@ extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const u
                                                    const uint16_t *A, const uint16_t *B, int32_t r, float s,
                                                    uint16_t *Y, uint16_t *sU_out, int32_t *dev_status,
                                                    qlora_stream_t stream) {
-  if (!W || !X || !A || !B || !Y || M <= 0 || W->rows <= 0 || W->cols <= 0) return QLORA_ERR_INVALID_ARG;
-  if (W->cols % qlora::kBlock || r < 8 || r > 64 || r % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (qlora::gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens: one launch, no scratch at all
-    return qlora::few_token_forward(W, X, M, A, B, r, s, Y, sU_out, stream);
-  // Scratch layout: [sU when the caller does not keep it][fp32 partial sums of s X A^T].
-  const size_t su_bytes = sU_out ? 0 : round_up_256(static_cast<size_t>(M) * static_cast<size_t>(r) * 2);
-  const size_t part_bytes = qlora::lora_rows_ws_floats(M, W->cols, r) * 4;
-  if (su_bytes + part_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;   // beyond the fixed maximum
+  // every argument is checked as qlora_linear_fwd checks it, before anything runs
+  qlora_status_t st = qlora::linear_fwd_check(W, X, M, A, B, r, s, Y, sU_out, dev_status);
+  if (st != QLORA_OK) return st;
+  const int64_t N = W->rows, K = W->cols;
+  const size_t need = qlora::linear_fwd_scratch_bytes(M, N, K, r, sU_out != nullptr);
+  if (need > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;   // beyond the fixed maximum
   void *scratch = nullptr;
-  qlora_status_t st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != QLORA_OK) return st;
   unsigned char *base = static_cast<unsigned char *>(scratch);
-  uint16_t *sU = sU_out ? sU_out : reinterpret_cast<uint16_t *>(base);
-  st = qlora_lora_xa(X, M, W->cols, A, r, s, sU, base + su_bytes, part_bytes, stream);
-  if (st != QLORA_OK) return st;
-  return qlora_fused_fwd(W, X, M, B, r, sU, Y, nullptr, 0, dev_status, stream);   // whole-tile schedule
+  if (M <= qlora::kSmallM)   // the few-token launch: all of its scratch
+    return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, nullptr, base, need, dev_status, stream);
+  // [sU when the caller does not keep it][the GEMM's stream-K partials, up to 64 tokens]
+  const size_t su_bytes = sU_out ? 0 : round_up_256(static_cast<size_t>(M) * static_cast<size_t>(r) * 2);
+  void *gemm_ws = M <= 64 ? static_cast<void *>(base + su_bytes) : nullptr;
+  return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, reinterpret_cast<uint16_t *>(base), gemm_ws,
+                               M <= 64 ? need - su_bytes : 0, dev_status, stream);
 }

@@ -75,10 +75,17 @@ cudaError_t launch_swiglu_pack_b(const uint16_t *Bg, const uint16_t *Bu, int64_t
                                  cudaStream_t st);
 cudaError_t launch_swiglu_unpack_db(const float *dBgu, int64_t F, int r, float *dBg, float *dBu, cudaStream_t st);
 
-// Few-token forward through the C-ABI types (validation + one launch).
-qlora_status_t few_token_forward(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
-                                 const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
-                                 qlora_stream_t stream);
+// The linear forward split into its validation (everything qlora_linear_fwd
+// checks before it launches anything), the scratch it needs when sU is or is
+// not kept by the caller, and the launches (see api.cu).
+qlora_status_t linear_fwd_check(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                                const uint16_t *B, int32_t r, float s, const uint16_t *Y, const uint16_t *sU_out,
+                                const int32_t *dev_status);
+size_t linear_fwd_scratch_bytes(int64_t M, int64_t N, int64_t K, int32_t r, bool keep_su);
+qlora_status_t linear_fwd_run(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
+                              const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
+                              uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes, int32_t *dev_status,
+                              qlora_stream_t stream);
 
 // Skinny LoRA products (fp32 accumulation).
 // out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if
@@ -96,6 +103,29 @@ size_t lora_rows_ws_floats(int64_t M, int64_t K, int r);
 size_t lora_cols_ws_floats(int64_t M, int64_t D, int r);
 
 int device_sm_count();
+
+// Token counts up to which the forward streams the weight (nf4_small_m.cu).
+constexpr int64_t kSmallM = 16;
+
+// Few-token forward (M <= 16) of one or more linears in one persistent launch
+// (see nf4_small_m.cu). Exactly one of A (the kernel then forms
+// sU = bf16(s X A^T), written to sU_out when given) and sU_in per linear.
+struct SmallProblem {
+  const uint8_t *codes;
+  const uint8_t *scale8;
+  const float *scale2;
+  int64_t N, K;
+  const uint16_t *X, *A, *B, *sU_in;
+  int r;
+  float s;
+  uint16_t *Y, *sU_out;
+};
+// Workspace bytes of launch_small_m for these linears (on the current device).
+size_t small_m_ws_bytes(const SmallProblem *pr, int count, int64_t M);
+// One launch per 16 linears, in order on `st`; with pdl the launch may start
+// streaming the weights before the preceding work on the stream has finished.
+cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *ws, bool pdl, int32_t *status,
+                           cudaStream_t st);
 
 // One CTA whose bounded mbarrier wait runs out (failure-path self-test).
 cudaError_t launch_bounded_wait_selftest(int32_t *status, cudaStream_t st);

@@ -163,9 +163,12 @@ qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r
  * X [M, K], A [r, K], B [N, r]: device bf16. Y [M, N]: device bf16, written.
  * sU_out [M, r]: device bf16 or NULL; if given, receives bf16_rn(s X A^T), the
  *   value the backward can reuse instead of recomputing it. For M <= 16 the
- *   forward is a single launch that forms sU itself (its fp32 sum runs in a
- *   different order than qlora_lora_xa's, so a backward that recomputes sU may
- *   see it differ by bf16 rounding) and the workspace is not touched.
+ *   forward is the single launch of qlora_linear_fwd_group for this one
+ *   linear: it forms sU itself (its fp32 sum runs in a different order than
+ *   qlora_lora_xa's, so a backward that recomputes sU may see it differ by
+ *   bf16 rounding) and applies each block constant to the block's partial
+ *   sum (Y then equals the definition up to the bf16 rounding of the levels,
+ *   within the same tolerance).
  * ws / ws_bytes: device workspace of at least qlora_linear_workspace() bytes.
  * dev_status: device int32 or NULL; set to QLORA_ERR_TIMEOUT if a bounded wait
  *   inside a kernel ran out (results are then incomplete). It is not cleared.
@@ -194,6 +197,63 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
                                 const uint16_t *dY, const uint16_t *sU, uint16_t *dX,
                                 float *dA, float *dB, void *ws, size_t ws_bytes,
                                 int32_t *dev_status, qlora_stream_t stream);
+
+/*
+ * Forward of several linears over the same few tokens in one launch, e.g. the
+ * query, key and value projections of one attention layer, or the gate and up
+ * projections of one MLP ("QLoRA and Fine-Tuning on One Consumer GPU", section
+ * "Where 24 GB goes": adapters on the attention and MLP projections; section
+ * "The idea in one line": each weight tile is dequantised to bf16 only for the
+ * moment it is used in a matmul).
+ * Each problem is one QLoRA linear with the arguments of qlora_linear_fwd:
+ *   Y = X W'^T + sU B^T,  sU = bf16_rn(s X A^T)  (written to sU_out if given).
+ * All problems of a call share the token count M, 1 <= M <= 16; X may be the
+ * same buffer for several problems. A few-token forward reads each packed
+ * weight once and does 2M flops per weight, so it is bound by memory and by
+ * the expansion of the codes, and one launch over the whole group keeps every
+ * SM streaming. The launch splits the (linear, 128-row tile, 64-weight block)
+ * work evenly over the SMs; the levels enter the tensor cores as
+ * bf16(1.43675 * level) with the block constant divided by 1.43675 applied to
+ * each block's fp32 partial sum, so Y equals the composite forward up to the
+ * bf16 rounding of the weights (within the GEMM tolerance of this library),
+ * and the result does not depend on timing.
+ * flags: 0, or QLORA_FWD_OVERLAP_PREVIOUS: the NF4 weights (codes, scale8,
+ *   scale2) are not written by the work queued before this call on the
+ *   stream, so the launch may begin streaming them before that work has
+ *   finished (programmatic dependent launch); X, A, B and the workspace are
+ *   still read only after it has finished.
+ * ws / ws_bytes: device workspace of at least qlora_linear_fwd_group_workspace()
+ *   bytes, 16-byte aligned. It needs no initialisation and the call leaves no
+ *   state the caller sees in it (a launch clears every flag it sets, so a
+ *   captured call can be replayed); one call at a time may use it. After a
+ *   QLORA_ERR_TIMEOUT in dev_status the workspace must be zero-filled (or
+ *   replaced) before it is used again.
+ * More than 16 problems run as consecutive launches of 16 on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (M > 16, or a shape qlora_linear_fwd
+ * rejects), MISALIGNED, WORKSPACE, CUDA; TIMEOUT in dev_status.
+ */
+typedef struct {
+  qlora_nf4_t W;           /* [N, K] NF4 weight (buffers on the device) */
+  const uint16_t *X;       /* [M, K] device bf16 */
+  const uint16_t *A;       /* [r, K] device bf16 */
+  const uint16_t *B;       /* [N, r] device bf16 */
+  int32_t r;               /* 8 <= r <= 64, r % 8 == 0 */
+  float s;                 /* alpha / r, finite */
+  uint16_t *Y;             /* [M, N] device bf16, written */
+  uint16_t *sU_out;        /* [M, r] device bf16 or NULL */
+} qlora_linear_problem_t;
+
+#define QLORA_FWD_OVERLAP_PREVIOUS 1
+
+/* Workspace bytes of qlora_linear_fwd_group for these problems on the current
+ * device (host; only the shapes, ranks and whether A and sU_out are given are
+ * read). Interface only: no passage of the pages defines it.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
+qlora_status_t qlora_linear_fwd_group_workspace(const qlora_linear_problem_t *problems, int32_t count,
+                                                int64_t M, size_t *bytes);
+qlora_status_t qlora_linear_fwd_group(const qlora_linear_problem_t *problems, int32_t count, int64_t M,
+                                      int32_t flags, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                      qlora_stream_t stream);
 
 /*
  * The five steps of the layer, one entry point each. qlora_linear_fwd runs
@@ -367,20 +427,28 @@ qlora_status_t qlora_lora_grads_adamw8(const uint16_t *X, const uint16_t *dY, in
  * inputs and outputs, a server whose device memory is all handed to a fixed
  * pool up front, code that must not call cudaMalloc between launches because
  * that call can synchronise the device).
- * It computes exactly what qlora_linear_fwd computes, with the same arguments
- * minus the workspace: its scratch (the split-K partial sums of s X A^T, plus
- * sU itself when sU_out is NULL) lives in one 8 MiB array compiled into the
- * library, which every GPU that loads the library holds until the process
- * exits. It calls no allocator.
- * Limit: round_up(M*r*2, 256) (only when sU_out is NULL) + the partial sums
- * (4 * splits * M * r bytes, splits <= 2 * SM count / ceil(M/64)) must fit in
- * 8 MiB; larger calls return QLORA_ERR_WORKSPACE before anything is launched.
+ * It validates its arguments exactly as qlora_linear_fwd does, before
+ * anything is launched, and then runs the same launches with the same
+ * schedule, so its results are bit for bit those of qlora_linear_fwd. Its
+ * scratch lives in one 8 MiB array compiled into the library, which every GPU
+ * that loads the library holds until the process exits; it calls no
+ * allocator. The scratch a call needs (it must fit in 8 MiB, else the call
+ * returns QLORA_ERR_WORKSPACE before anything is launched):
+ *   M <= 16:       the few-token launch's flags, partial tiles (SM count x 128
+ *                  rows x 8 or 16 tokens x 4 bytes), pieces of s X A^T and, when
+ *                  sU_out is NULL, sU: about 0.6 to 1.3 MB;
+ *   16 < M <= 64:  round_up(M*r*2, 256) when sU_out is NULL, plus the fused
+ *                  GEMM's stream-K partials (SM count x 128 x 64 x 4 bytes,
+ *                  about 4.9 MB on 148 SMs);
+ *   M > 64:        round_up(M*r*2, 256) when sU_out is NULL, nothing otherwise.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture. Every call shares the one array and leaves its contents
- * behind; nothing in it needs to start at zero, but calls whose kernels can
- * overlap on the GPU (other streams, other host threads) race on it, so the
- * caller must serialise them.
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture. The cached address belongs to the
+ * device's context: after cudaDeviceReset on a device this call must not be
+ * used on that device again in the same process. Every call shares the one
+ * array and leaves its contents behind; nothing in it needs to start at zero,
+ * but calls whose kernels can overlap on the GPU (other streams, other host
+ * threads) race on it, so the caller must serialise them.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA.
  */
 qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const uint16_t *X, int64_t M,
