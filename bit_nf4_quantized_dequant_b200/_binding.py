@@ -256,8 +256,8 @@ def linear_workspace(M: int, N: int, K: int, r: int) -> int:
 def _ws(ws, M, N, K, r, device):
     import torch
     need = linear_workspace(M, N, K, r)
-    if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    if ws is None:   # the first bytes (a counter page) must be zero before first use
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
     return ws
 
 
@@ -338,7 +338,7 @@ def linear_fwd_group(problems, ws=None, flags: int = 0, status=None, stream=None
     if arr is None:
         arr = _problem_array(problems)
     if ws is None:
-        ws = torch.empty(linear_fwd_group_workspace(problems, M), dtype=torch.uint8, device=problems[0].X.device)
+        ws = torch.zeros(linear_fwd_group_workspace(problems, M), dtype=torch.uint8, device=problems[0].X.device)
     _check(library().qlora_linear_fwd_group(arr, len(problems), M, flags, _ptr(ws), ws.numel(), _ptr(status),
                                             _stream(stream)), "qlora_linear_fwd_group")
     return [p.Y for p in problems]

@@ -78,36 +78,39 @@ static size_t small_fused_ws_bytes(int64_t M) {
   return small_m_ws_bytes(&p, 1, M);
 }
 
-// The optional workspace of qlora_fused_fwd / qlora_fused_dx: the stream-K
-// partials of the GEMM, or for a few tokens the persistent forward's.
+// The optional workspace of qlora_fused_fwd / qlora_fused_dx: the few-token
+// launch's counter page, then the stream-K partials of the GEMM or, for a few
+// tokens, the persistent forward's partials.
 static size_t fused_ws_bytes(int64_t M) {
   const size_t g = fused_gemm_ws_bytes(M);
-  if (M > kSmallM) return g;
+  if (M > kSmallM) return kSmallCounterBytes + g;
   const size_t sm = small_fused_ws_bytes(M);
-  return sm > g ? sm : g;
+  return kSmallCounterBytes + (sm > g ? sm : g);
 }
 
 // Workspace layout of the linear calls (offsets in bytes, 256-byte aligned):
+//   [counter page of the few-token forward (zero between calls)]
 //   [sU scratch: M*r bf16][sT: M*r bf16][fp32 partial sums of the skinny products]
-//   [stream-K workspace of the fused GEMMs]
+//   [stream-K workspace of the fused GEMMs, or the few-token forward's partials]
 struct WsLayout {
-  size_t su, st, part, part_floats, gemm, gemm_bytes, total;
+  size_t cnt, su, st, part, part_floats, gemm, gemm_bytes, total;
 };
 
 static WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r) {
   WsLayout w{};
   const size_t mr = round_up(static_cast<size_t>(M) * r * 2, 256);
-  w.su = 0;
-  w.st = mr;
-  w.part = 2 * mr;
+  w.cnt = 0;
+  w.su = kSmallCounterBytes;
+  w.st = w.su + mr;
+  w.part = w.st + mr;
   size_t f = lora_rows_ws_floats(M, K, r);
   f = f > lora_rows_ws_floats(M, N, r) ? f : lora_rows_ws_floats(M, N, r);
   f = f > lora_cols_ws_floats(M, K, r) ? f : lora_cols_ws_floats(M, K, r);
   f = f > lora_cols_ws_floats(M, N, r) ? f : lora_cols_ws_floats(M, N, r);
   w.part_floats = f;
   w.gemm = w.part + round_up(f * 4, 256);
-  w.gemm_bytes = fused_gemm_ws_bytes(M);
-  if (M <= kSmallM) {   // the few-token forward uses this region instead
+  w.gemm_bytes = fused_ws_bytes(M);   // the workspace of qlora_fused_fwd / qlora_fused_dx
+  if (M <= kSmallM) {   // the few-token forward uses this region instead (with the page at w.cnt)
     const size_t sm = small_fwd_ws_bytes(M, N, K, r);
     w.gemm_bytes = sm > w.gemm_bytes ? sm : w.gemm_bytes;
   }
@@ -160,10 +163,10 @@ size_t linear_fwd_scratch_bytes(int64_t M, int64_t N, int64_t K, int32_t r, bool
     p.r = r;
     p.A = reinterpret_cast<const uint16_t *>(16);
     p.sU_out = keep_su ? reinterpret_cast<uint16_t *>(16) : nullptr;
-    return small_m_ws_bytes(&p, 1, M);
+    return kSmallCounterBytes + small_m_ws_bytes(&p, 1, M);
   }
-  size_t b = keep_su ? 0 : round_up(static_cast<size_t>(M) * r * 2, 256);
-  if (M <= 64) b += round_up(fused_gemm_ws_bytes(M), 256);   // the stream-K schedule of short token tiles
+  size_t b = kSmallCounterBytes + (keep_su ? 0 : round_up(static_cast<size_t>(M) * r * 2, 256));
+  if (M <= 64) b += round_up(fused_ws_bytes(M), 256);   // the stream-K schedule of short token tiles
   return b;
 }
 
@@ -172,8 +175,8 @@ size_t linear_fwd_scratch_bytes(int64_t M, int64_t N, int64_t K, int32_t r, bool
 // the few-token launch's (M <= kSmallM).
 qlora_status_t linear_fwd_run(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
                               const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
-                              uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes, int32_t *dev_status,
-                              qlora_stream_t stream) {
+                              void *counters, uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes,
+                              int32_t *dev_status, qlora_stream_t stream) {
   const int64_t N = W->rows, K = W->cols;
   if (M <= kSmallM) {
     SmallProblem p{};
@@ -190,7 +193,8 @@ qlora_status_t linear_fwd_run(const qlora_nf4_t *W, const uint16_t *X, int64_t M
     p.Y = Y;
     p.sU_out = sU_out;
     if (!gemm_ws || gemm_ws_bytes < small_m_ws_bytes(&p, 1, M)) return QLORA_ERR_WORKSPACE;
-    return cuda_status(launch_small_m(&p, 1, M, gemm_ws, false, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(
+        launch_small_m(&p, 1, M, gemm_ws, counters, false, dev_status, reinterpret_cast<cudaStream_t>(stream)));
   }
   uint16_t *sU = sU_out ? sU_out : su_scratch;
   qlora_status_t st = qlora_lora_xa(X, M, K, A, r, s, sU, nullptr, 0, stream);
@@ -361,7 +365,7 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
   g.lora_act = lora_act;
   g.out = out;
   g.dev_status = dev_status;
-  g.ws = ws;
+  g.ws = ws ? static_cast<uint8_t *>(ws) + kSmallCounterBytes : nullptr;
   if (mode == 0 && M <= kSmallM && ws && W->rows <= INT32_MAX && W->cols <= INT32_MAX) {
     // a few tokens with a workspace: the persistent weight-streaming launch
     SmallProblem p{};
@@ -375,7 +379,8 @@ static qlora_status_t fused(int mode, const qlora_nf4_t *W, const uint16_t *act,
     p.sU_in = lora_act;
     p.r = r;
     p.Y = out;
-    return cuda_status(launch_small_m(&p, 1, M, ws, false, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_small_m(&p, 1, M, static_cast<uint8_t *>(ws) + kSmallCounterBytes, ws, false,
+                                      dev_status, reinterpret_cast<cudaStream_t>(stream)));
   }
   if (mode == 0 && gemv_fwd_supported(W->rows, W->cols, M))   // a few tokens, no workspace: one cluster launch
     return cuda_status(launch_nf4_gemv_fwd(W->codes, W->scale8, W->scale2, W->rows, W->cols, M, act, lora_w,
@@ -452,8 +457,8 @@ qlora_status_t qlora_linear_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
   if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
-  return linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, reinterpret_cast<uint16_t *>(wsb + L.su), wsb + L.gemm,
-                        L.gemm_bytes, dev_status, stream);
+  return linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, wsb + L.cnt, reinterpret_cast<uint16_t *>(wsb + L.su),
+                        wsb + L.gemm, L.gemm_bytes, dev_status, stream);
 }
 
 qlora_status_t qlora_linear_fwd_group_workspace(const qlora_linear_problem_t *problems, int32_t count, int64_t M,
@@ -471,7 +476,7 @@ qlora_status_t qlora_linear_fwd_group_workspace(const qlora_linear_problem_t *pr
     pr[i].A = q.A;
     pr[i].sU_out = q.sU_out;
   }
-  *bytes = small_m_ws_bytes(pr.data(), count, M);
+  *bytes = kSmallCounterBytes + small_m_ws_bytes(pr.data(), count, M);
   return QLORA_OK;
 }
 
@@ -500,9 +505,10 @@ qlora_status_t qlora_linear_fwd_group(const qlora_linear_problem_t *problems, in
     p.Y = q.Y;
     p.sU_out = q.sU_out;
   }
-  if (!ws || ws_bytes < small_m_ws_bytes(pr.data(), count, M)) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < kSmallCounterBytes + small_m_ws_bytes(pr.data(), count, M)) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_MISALIGNED;
-  return cuda_status(launch_small_m(pr.data(), count, M, ws, (flags & QLORA_FWD_OVERLAP_PREVIOUS) != 0, dev_status,
+  return cuda_status(launch_small_m(pr.data(), count, M, static_cast<uint8_t *>(ws) + kSmallCounterBytes, ws,
+                                    (flags & QLORA_FWD_OVERLAP_PREVIOUS) != 0, dev_status,
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -31,9 +31,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per device
 constexpr int kMaxDevices = 64;
 }  // namespace
 
-// The shared scratch. Nothing in it has to start at zero: each call writes
-// every byte it later reads, and the counters of the few-token launch carry a
-// per-launch value that makes stale contents count as zero.
+// The shared scratch. Its first 256 bytes are the few-token launch's counter
+// page: zero at load (a __device__ array is zero-initialised) and left zero by
+// every call that completes; every other byte a call reads it writes first.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -73,12 +73,15 @@ extern "C" qlora_status_t qlora_linear_fwd_noalloc(const qlora_nf4_t *W, const u
   void *scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != QLORA_OK) return st;
-  unsigned char *base = static_cast<unsigned char *>(scratch);
-  if (M <= qlora::kSmallM)   // the few-token launch: all of its scratch
-    return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, nullptr, base, need, dev_status, stream);
+  // [the few-token launch's counter page, zero between calls][the rest]
+  unsigned char *cnt = static_cast<unsigned char *>(scratch);
+  unsigned char *base = cnt + qlora::kSmallCounterBytes;
+  const size_t rest = need - qlora::kSmallCounterBytes;
+  if (M <= qlora::kSmallM)   // the few-token launch: its partials and pieces of s X A^T
+    return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, cnt, nullptr, base, rest, dev_status, stream);
   // [sU when the caller does not keep it][the GEMM's stream-K partials, up to 64 tokens]
   const size_t su_bytes = sU_out ? 0 : round_up_256(static_cast<size_t>(M) * static_cast<size_t>(r) * 2);
   void *gemm_ws = M <= 64 ? static_cast<void *>(base + su_bytes) : nullptr;
-  return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, reinterpret_cast<uint16_t *>(base), gemm_ws,
-                               M <= 64 ? need - su_bytes : 0, dev_status, stream);
+  return qlora::linear_fwd_run(W, X, M, A, B, r, s, Y, sU_out, cnt, reinterpret_cast<uint16_t *>(base), gemm_ws,
+                               M <= 64 ? rest - su_bytes : 0, dev_status, stream);
 }

@@ -84,8 +84,8 @@ qlora_status_t linear_fwd_check(const qlora_nf4_t *W, const uint16_t *X, int64_t
 size_t linear_fwd_scratch_bytes(int64_t M, int64_t N, int64_t K, int32_t r, bool keep_su);
 qlora_status_t linear_fwd_run(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *A,
                               const uint16_t *B, int32_t r, float s, uint16_t *Y, uint16_t *sU_out,
-                              uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes, int32_t *dev_status,
-                              qlora_stream_t stream);
+                              void *counters, uint16_t *su_scratch, void *gemm_ws, size_t gemm_ws_bytes,
+                              int32_t *dev_status, qlora_stream_t stream);
 
 // Skinny LoRA products (fp32 accumulation).
 // out[m, j] = bf16_rn(s * sum_k Z[m, k] * Wl(j, k)); Wl(j, k) = W[j*K + k] if
@@ -120,12 +120,15 @@ struct SmallProblem {
   float s;
   uint16_t *Y, *sU_out;
 };
-// Workspace bytes of launch_small_m for these linears (on the current device).
+// Workspace bytes of launch_small_m for these linears (on the current device),
+// besides its counter page: kSmallCounterBytes that must be zero before the
+// first launch and that every launch leaves zero (nothing else may write them).
+constexpr size_t kSmallCounterBytes = 256;
 size_t small_m_ws_bytes(const SmallProblem *pr, int count, int64_t M);
-// One launch per 16 linears, in order on `st`; with pdl the launch may start
+// One launch per 8 linears, in order on `st`; with pdl the launch may start
 // streaming the weights before the preceding work on the stream has finished.
-cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *ws, bool pdl, int32_t *status,
-                           cudaStream_t st);
+cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *ws, void *counters, bool pdl,
+                           int32_t *status, cudaStream_t st);
 
 // One CTA whose bounded mbarrier wait runs out (failure-path self-test).
 cudaError_t launch_bounded_wait_selftest(int32_t *status, cudaStream_t st);

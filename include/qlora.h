@@ -152,9 +152,13 @@ qlora_status_t qlora_dqfp8_dequantize(const qlora_nf4_t *q, uint16_t *out, qlora
  * of the pages defines it; it exists because this library never allocates, so
  * the caller sizes and owns the scratch memory the kernels use. It takes
  * (M, N, K, r) rather than the weight itself so that a caller can size the
- * workspace before any weight is quantised. The same workspace may be reused
- * by consecutive calls on one stream; calls that run concurrently need
- * separate workspaces. Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
+ * workspace before any weight is quantised. The workspace starts with a
+ * 256-byte counter page that must be zero before the workspace is first used
+ * (e.g. one cudaMemsetAsync of the whole buffer); every call that completes
+ * without a device error leaves the page zero, and the rest of the workspace
+ * needs no initialisation. The same workspace may be reused by consecutive
+ * calls on one stream; calls that run concurrently need separate workspaces.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE. */
 qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r,
                                       size_t *bytes);
 
@@ -169,7 +173,8 @@ qlora_status_t qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r
  *   bf16 rounding) and applies each block constant to the block's partial
  *   sum (Y then equals the definition up to the bf16 rounding of the levels,
  *   within the same tolerance).
- * ws / ws_bytes: device workspace of at least qlora_linear_workspace() bytes.
+ * ws / ws_bytes: device workspace of at least qlora_linear_workspace() bytes
+ *   (its first 256 bytes zero before first use, see there).
  * dev_status: device int32 or NULL; set to QLORA_ERR_TIMEOUT if a bounded wait
  *   inside a kernel ran out (results are then incomplete). It is not cleared.
  * Supported: M >= 1, N % 16 == 0, K % 64 == 0, r % 8 == 0 with 8 <= r <= 64,
@@ -223,12 +228,12 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
  *   finished (programmatic dependent launch); X, A, B and the workspace are
  *   still read only after it has finished.
  * ws / ws_bytes: device workspace of at least qlora_linear_fwd_group_workspace()
- *   bytes, 16-byte aligned. It needs no initialisation and the call leaves no
- *   state the caller sees in it (a launch clears every flag it sets, so a
+ *   bytes, 16-byte aligned, zero-filled before its first use. Every call leaves
+ *   it as it found it (a launch resets each counter and flag it sets, so a
  *   captured call can be replayed); one call at a time may use it. After a
  *   QLORA_ERR_TIMEOUT in dev_status the workspace must be zero-filled (or
  *   replaced) before it is used again.
- * More than 16 problems run as consecutive launches of 16 on `stream`.
+ * More than 8 problems run as consecutive launches of 8 on `stream`.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (M > 16, or a shape qlora_linear_fwd
  * rejects), MISALIGNED, WORKSPACE, CUDA; TIMEOUT in dev_status.
  */
@@ -287,9 +292,12 @@ qlora_status_t qlora_fused_workspace(int64_t M, size_t *bytes);
  *   workspace and M <= 64 (where whole tiles would leave most SMs idle) the
  *   (tile, K-step) work is split evenly over all SMs and tiles cut between CTAs
  *   are summed through fp32 partials kept there (results equal up to fp32
- *   rounding order); larger M keeps whole tiles. The workspace needs no
- *   initialisation and keeps no state the caller sees; one launch at a time may
- *   use a given workspace.
+ *   rounding order); for M <= 16 the forward is the persistent few-token
+ *   launch of qlora_linear_fwd_group; larger M keeps whole tiles. The first
+ *   256 bytes of the workspace are a counter page that must be zero before
+ *   first use and that every call leaves zero; the rest needs no
+ *   initialisation and keeps no state the caller sees; one launch at a time
+ *   may use a given workspace.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
 qlora_status_t qlora_fused_fwd(const qlora_nf4_t *W, const uint16_t *X, int64_t M, const uint16_t *B,
                                int32_t r, const uint16_t *sU, uint16_t *Y, void *ws, size_t ws_bytes,
@@ -434,12 +442,13 @@ qlora_status_t qlora_lora_grads_adamw8(const uint16_t *X, const uint16_t *dY, in
  * that loads the library holds until the process exits; it calls no
  * allocator. The scratch a call needs (it must fit in 8 MiB, else the call
  * returns QLORA_ERR_WORKSPACE before anything is launched):
+ * always a 256-byte counter page, and
  *   M <= 16:       the few-token launch's flags, partial tiles (SM count x 128
  *                  rows x 8 or 16 tokens x 4 bytes), pieces of s X A^T and, when
  *                  sU_out is NULL, sU: about 0.6 to 1.3 MB;
  *   16 < M <= 64:  round_up(M*r*2, 256) when sU_out is NULL, plus the fused
- *                  GEMM's stream-K partials (SM count x 128 x 64 x 4 bytes,
- *                  about 4.9 MB on 148 SMs);
+ *                  GEMM's workspace (qlora_fused_workspace(M), about 4.9 MB on
+ *                  148 SMs);
  *   M > 64:        round_up(M*r*2, 256) when sU_out is NULL, nothing otherwise.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current and caches it; make that

@@ -125,7 +125,7 @@ def test_fused_equals_gradients_then_step(lib):
     # separate
     dA = torch.empty((r, K), dtype=torch.float32, device="cuda")
     dB = torch.empty((N, r), dtype=torch.float32, device="cuda")
-    ws = torch.empty(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
     lib.lora_grads(X, dY, sU, sT, dA, dB, ws)
     Am2, Bm2 = A0.clone(), B0.clone()
     Ab2 = torch.empty(K * r, dtype=torch.bfloat16, device="cuda")

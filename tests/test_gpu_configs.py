@@ -223,7 +223,7 @@ def test_mlp_7b_chain_fused_swiglu(lib, mlp_7b):
     Agu = to_dev_bf16(np.concatenate([cg["A"], cu["A"]]))
     Bgu = lib.swiglu_pack_b(to_dev_bf16(cg["B"]), to_dev_bf16(cu["B"]))
     Ad, Bd = to_dev_bf16(cd["A"]), to_dev_bf16(cd["B"])
-    ws = torch.empty(lib.linear_workspace(M, 2 * Fd, K, 2 * r), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_workspace(M, 2 * Fd, K, 2 * r), dtype=torch.uint8, device="cuda")
     sUgu = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
     lib.lora_xa(X, Agu, s, sUgu, ws)
     h = lib.swiglu_fwd(qgu, X, Bgu, sUgu)

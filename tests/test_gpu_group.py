@@ -110,7 +110,7 @@ def test_group_graph_replay_with_changing_inputs(lib):
     import torch
     shapes = [(512, 2048, 16), (256, 2048, 16)]
     probs, _ = _group(lib, shapes, 8, shared_x=True)
-    ws = torch.empty(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
     arr = lib._binding._problem_array(probs)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
@@ -142,7 +142,7 @@ def test_group_overlap_flag_sees_the_preceding_kernel(lib):
     shapes = [(1024, 1024, 16), (256, 1024, 16)]
     probs, refs = _group(lib, shapes, 8, shared_x=True)
     X_true = probs[0].X.clone()
-    ws = torch.empty(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
     for _ in range(3):
         probs[0].X.zero_()
         torch.cuda.synchronize()
@@ -155,7 +155,7 @@ def test_group_overlap_flag_sees_the_preceding_kernel(lib):
 def test_group_rejects_bad_arguments(lib):
     import torch
     probs, _ = _group(lib, [(128, 256, 16)], 8)
-    ws = torch.empty(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_fwd_group_workspace(probs, 8), dtype=torch.uint8, device="cuda")
     arr = lib._binding._problem_array(probs)
     L = lib.library()
     st = lambda **kw: L.qlora_linear_fwd_group(arr, kw.get("count", 1), kw.get("M", 8), kw.get("flags", 0),

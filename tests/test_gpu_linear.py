@@ -151,10 +151,11 @@ def test_fused_gemm_whole_tile_and_stream_k(lib, N, K, M, r):
     T = h["dY"] @ h["B"]
     sU = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
     sT = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
-    lws = torch.empty(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    lws = torch.zeros(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
     lib.lora_xa(d["X"], d["A"], s, sU, lws)
     lib.lora_dyb(d["dY"], d["B"], s, sT, lws)
     gws = torch.full((lib.fused_workspace(M),), 0xAB, dtype=torch.uint8, device="cuda")
+    gws[:256].zero_()   # the counter page starts at zero; the rest needs no initialisation
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = {}
     for name, ws, schedule in (("auto", None, lib.SCHEDULE_AUTO), ("single", None, lib.SCHEDULE_SINGLE),
@@ -182,8 +183,8 @@ def test_stream_k_graph_replays(lib):
     N, K, M, r, s = 2048, 512, 40, 16, 2.0
     h, d = _setup(lib, N, K, M, r, index=6)
     sU = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
-    lws = torch.empty(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
-    gws = torch.empty(lib.fused_workspace(M), dtype=torch.uint8, device="cuda")
+    lws = torch.zeros(lib.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+    gws = torch.zeros(lib.fused_workspace(M), dtype=torch.uint8, device="cuda")
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     X = d["X"].clone()
     lib.lora_xa(X, d["A"], s, sU, lws)

@@ -55,7 +55,7 @@ def test_swiglu_fused_forward_and_backward(lib, F, K, M, r):
     Xd, dHd = to_dev_bf16(X), to_dev_bf16(dH)
     Agu = to_dev_bf16(np.concatenate([Ag, Au]))
     Bgu = lib.swiglu_pack_b(to_dev_bf16(Bg), to_dev_bf16(Bu))
-    ws = torch.empty(lib.linear_workspace(M, 2 * F, K, 2 * r), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.linear_workspace(M, 2 * F, K, 2 * r), dtype=torch.uint8, device="cuda")
     sUgu = torch.empty((M, 2 * r), dtype=torch.bfloat16, device="cuda")
     lib.lora_xa(Xd, Agu, s, sUgu, ws)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -66,10 +66,12 @@ def test_noalloc_forward_matches_oracle_and_workspace_forward(lib, M):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
-    """Just over the limit: 65,600 tokens at rank 64 without a caller-kept sU
-    need round_up(65600 * 64 * 2, 256) = 8,396,800 bytes of scratch > 8 MiB.
-    Every pointer is a real device buffer, so even a regression that launched
-    would compute on valid memory; the call must refuse before launching."""
+    """Just over the limit: beyond 16 tokens and at more than 64 the scratch
+    is the 256-byte counter page plus round_up(M * r * 2, 256) for sU when the
+    caller does not keep it. 65,600 tokens at rank 64 need 8,397,056 bytes >
+    8 MiB; 65,534 tokens need exactly 8 MiB. Every pointer is a real device
+    buffer, so even a regression that launched would compute on valid memory;
+    the call must refuse before launching."""
     import torch
     N = K = 1024
     M, r = 65600, 64
@@ -82,8 +84,8 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     assert _call_noalloc(lib, q, X, A, B, r, 2.0, Y, None) == 4   # QLORA_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert bool((Y[:: 4099] == 7.0).all())                        # nothing was written
-    # one token fewer per 64 rows fits: M = 65536 needs exactly 8 MiB
-    assert _call_noalloc(lib, q, X, A, B, r, 2.0, Y, None, M=65536) == 0
+    assert _call_noalloc(lib, q, X, A, B, r, 2.0, Y, None, M=65535) == 4
+    assert _call_noalloc(lib, q, X, A, B, r, 2.0, Y, None, M=65534) == 0
     torch.cuda.synchronize()
 
 
