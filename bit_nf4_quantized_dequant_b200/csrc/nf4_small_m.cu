@@ -62,6 +62,7 @@
 // found it, and a captured launch can be replayed.
 #include <atomic>
 #include <chrono>
+#include <cstring>
 
 #include "qlora_device.cuh"
 
@@ -69,16 +70,20 @@ namespace qlora {
 
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+bool encode_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, const uint64_t dims[3],
+               const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
 
 namespace {
 
 constexpr int kSmMaxProblems = 8;
 constexpr int kSmTileRows = 128;
 constexpr int kConsumerWarps = 8;                    // 4 row groups x 2 K slices
-constexpr int kProducerWarp = 8;
-constexpr int kEpiWarp0 = 9;
+constexpr int kProducerWarp = 8;                     // the copies of codes and activations
+constexpr int kScaleWarp0 = 9;                       // the block scales: rows 0-63 and 64-127
+constexpr int kScaleWarps = 2;
+constexpr int kEpiWarp0 = kScaleWarp0 + kScaleWarps;
 constexpr int kEpiWarps = 4;
-constexpr int kSmThreads = (kEpiWarp0 + kEpiWarps) * 32;   // 416
+constexpr int kSmThreads = (kEpiWarp0 + kEpiWarps) * 32;   // 480
 constexpr int kChunkBlocks = 8;                      // NF4 blocks (of 64 weights) per chunk
 constexpr uint32_t kCodeSlot = kSmTileRows * kChunkBlocks * 32;   // 32 KB of codes per chunk
 constexpr int kUnitK = 128;                          // K per piece of X A^T (two NF4 blocks)
@@ -87,8 +92,7 @@ constexpr int kMaxSlots = 3;
 constexpr float kLambda = 1.43675f;
 constexpr float kInvLambda = 1.0f / 1.43675f;
 constexpr uint32_t kEpiBar = 1;                      // named barrier of the epilogue warps
-
-__constant__ float c_levels[16] = QLORA_NF4_LEVELS;
+constexpr uint32_t kTableBar = 2;                    // named barrier of the consumer warps
 
 struct SmProblem {
   const uint8_t *codes;
@@ -106,20 +110,34 @@ struct SmProblem {
   float s;
 };
 
-struct SmParams {
-  CUtensorMap tm_codes[kSmMaxProblems];   // codes of each linear as u8 [N][K/2], 128 x 128-byte boxes, swizzled
-  CUtensorMap tm_x[kSmMaxProblems];       // activations as bf16 [M][K], boxes of MP tokens x 256
+// What the kernel reads besides the tensor maps; copied into shared memory
+// at the start of a launch by all threads at once (one round of parameter
+// loads instead of a chain of dependent ones).
+struct __align__(16) SmHead {
   SmProblem p[kSmMaxProblems];
   int32_t count, M;
   int64_t w_units;
   int32_t u_units;
+  int32_t pdl;
+  int32_t x3d;             // tm_x is the 3-D map (one box per chunk), else one 2-D box per block
+  int32_t rawtma;          // raw constants by TMA (tm_q8, tm_s2), else by cp.async
+  int32_t pad_[2];
   uint64_t epoch;          // launch value, 1 <= epoch < 2^44
-  uint64_t *flags;         // [grid]: a contributor's partial is published
+  uint64_t *flags;         // [grid]: a contributor's partial is published; then [count]: sU ready
   float *slots;            // [grid][MP][128]: published partials
   unsigned long long *ucnt;    // [count]: pieces of X A^T done (zero at launch)
   unsigned long long *ucons;   // [count]: tiles that have used them (zero at launch)
   int32_t *status;
-  int32_t pdl;
+  uint16_t lvl[16];        // bf16(lambda * level[i])
+};
+static_assert(sizeof(SmHead) % 16 == 0, "copied as 16-byte words");
+
+struct SmParams {
+  CUtensorMap tm_codes[kSmMaxProblems];   // codes of each linear as u8 [N][K/2], 128 x 128-byte boxes, swizzled
+  CUtensorMap tm_x[kSmMaxProblems];       // activations as bf16 [M][K]: boxes [8 blocks][MP tokens][64], swizzled
+  CUtensorMap tm_q8[kSmMaxProblems];      // first-level constants as u8 [N][K/64], boxes 16 x 128
+  CUtensorMap tm_s2[kSmMaxProblems];      // second-level constants as f32 [1][groups], boxes of 256
+  SmHead h;
 };
 
 // ---- small PTX helpers ------------------------------------------------------
@@ -130,10 +148,6 @@ __device__ __forceinline__ void cp_async_8(uint32_t saddr, const void *g) {
 }
 __device__ __forceinline__ void cp_async_4(uint32_t saddr, const void *g, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(saddr), "l"(g), "r"(src_bytes) : "memory");
-}
-// One arrival on `bar` once this thread's earlier cp.async copies are done.
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
   uint32_t v;
@@ -210,7 +224,7 @@ __device__ __forceinline__ bool wait_word(const uint64_t *w, uint64_t v, volatil
 }
 
 // ---- the unit list ----------------------------------------------------------
-__device__ __forceinline__ int problem_of(const SmParams &P, int64_t u) {
+__device__ __forceinline__ int problem_of(const SmHead &P, int64_t u) {
   int p = 0;
 #pragma unroll 1
   for (int i = 1; i < P.count; ++i)
@@ -243,7 +257,7 @@ __device__ __forceinline__ void walk_init(Walk &w, int64_t ub, int64_t ue) {
 }
 
 template <int C>
-__device__ __forceinline__ bool walk_next(const SmParams &P, Walk &w, Chunk &c) {
+__device__ __forceinline__ bool walk_next(const SmHead &P, Walk &w, Chunk &c) {
   if (w.kb >= w.kb_hi) {
     if (w.u >= w.ue) return false;
     const int p = problem_of(P, w.u);
@@ -273,222 +287,367 @@ __device__ __forceinline__ bool walk_next(const SmParams &P, Walk &w, Chunk &c) 
 }
 
 // ---- shared-memory layout -----------------------------------------------------
-// [level table 64 KB][codes ring][activation ring][constants ring][epilogue
-// buffers][sU][partial sums][barriers], from the start of dynamic shared memory.
+// The level table sits at a 64 KB-aligned shared address, so that one PRMT
+// forms a lookup's whole address (table | byte << 8 | lane * 4). Its entries
+// use the first 128 bytes of every 256; the second halves hold the epilogue
+// buffers (byte o of them at lut + 256 (o >> 7) + 128 + (o & 127)). The space
+// between the start of dynamic shared memory and the table takes the rings of
+// activations, block scales and raw constants, sU and the barriers, or, if
+// they do not fit there, goes after the code ring.
 template <int MP>
 struct Layout {
   static constexpr int C = kChunkBlocks;
   static constexpr int NS = MP == 8 ? 3 : 2;                // ring depth
-  static constexpr uint32_t XBOX = MP * 512;                // one TMA box: MP tokens x 256 bf16
-  static constexpr uint32_t XSLOT = 2 * XBOX;               // a chunk's 512 K
-  static constexpr uint32_t SSLOT = kSmTileRows * 8 + kSmTileRows * 8;   // q8 [128][8 B], (d_a, d_b) [128]
+  static constexpr uint32_t XBOX = MP * 128;                // a block of MP tokens: [token][64 bf16], 128-byte swizzle
+  static constexpr uint32_t XSLOT = C * XBOX;               // a chunk's 512 K
+  static constexpr uint32_t SCSLOT = C * kSmTileRows * 4;   // block scales [block][row group][g][4] floats
+  static constexpr uint32_t RAWQ8 = kSmTileRows * 16;       // raw q8: [row][16 B], the chunk's 8 at byte kbA % 16
+  static constexpr uint32_t RAWSLOT = RAWQ8 + 1024;         // then 256 second-level constants, or (d_a, d_b) per row
   static constexpr uint32_t EROW = MP;                      // floats per row of an epilogue buffer
   static constexpr uint32_t EBUF = 2 * kSmTileRows * EROW * 4;   // [slice][row][token]
+  static_assert(2 * EBUF <= kLutBytes / 2, "epilogue buffers fit the table's second halves");
   static constexpr uint32_t SUBYTES = MP * 64 * 4;          // sU of one linear as float [t][64]
-  static constexpr uint32_t REDBYTES = 128 * 16;            // partial sums of the pieces of X A^T
-  static constexpr uint32_t BARBYTES = 128;
-  static constexpr uint32_t CRING = kLutBytes;
-  static constexpr uint32_t XRING = CRING + NS * kCodeSlot;
-  static constexpr uint32_t SRING = XRING + NS * XSLOT;
-  static constexpr uint32_t EBUFS = SRING + NS * SSLOT;
-  static constexpr uint32_t SUS = EBUFS + 2 * EBUF;
-  static constexpr uint32_t REDS = SUS + SUBYTES;
-  static constexpr uint32_t BARS = REDS + REDBYTES;
-  static constexpr uint32_t END = BARS + BARBYTES + 16;
-  static constexpr uint32_t request() { return END; }
+  static constexpr uint32_t BARBYTES = 256;
+  static constexpr uint32_t S_X = 0;
+  static constexpr uint32_t S_SC = S_X + NS * XSLOT;
+  static constexpr uint32_t S_RAW = S_SC + NS * SCSLOT;
+  static constexpr uint32_t S_SU = S_RAW + NS * RAWSLOT;
+  static constexpr uint32_t S_BAR = S_SU + SUBYTES;
+  static constexpr uint32_t G1 = S_BAR + BARBYTES + 16;
+  static constexpr uint32_t CODES = NS * kCodeSlot;
+  // bytes used from the start of dynamic shared memory at shared address
+  // `base`; the small regions start on a 1 KB boundary (swizzled TMA boxes)
+  static constexpr uint32_t extent(uint32_t base) {
+    const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu, avail = lut - ((base + 1023u) & ~1023u);
+    return lut - base + kLutBytes + CODES + (G1 <= avail ? 0 : G1);
+  }
+  // dynamic shared memory to request: the largest extent over the starts
+  // this kernel can see (16-byte aligned, at most 4 KB)
+  static constexpr uint32_t request() {
+    uint32_t m = 0;
+    for (uint32_t b = 0; b <= 4096; b += 16) m = extent(b) > m ? extent(b) : m;
+    return m;
+  }
 };
+static_assert(Layout<8>::request() <= 232448 && Layout<16>::request() <= 232448, "shared memory");
 
 template <int NT>
-__global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid_constant__ SmParams P) {
+__global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid_constant__ SmParams Pk) {
   constexpr int MP = 8 * NT;
   using L = Layout<MP>;
   constexpr int C = L::C;
   constexpr int NS = L::NS;
   constexpr int D = C / 2;   // own blocks of a consumer warp per chunk
   extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ SmHead s_head;
+  const SmHead &P = s_head;
 
-  if (P.pdl) grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
 
+  // ---- layout --------------------------------------------------------------
   const uint32_t base = smem_u32(smem);
   uint8_t *gbase = smem - base;   // generic pointer of shared address 0 (for plain C++ accesses)
-  const uint32_t lut = base, cring = base + L::CRING, xring = base + L::XRING, sring = base + L::SRING;
-  const uint32_t ebuf = base + L::EBUFS, sus = base + L::SUS, reds = base + L::REDS, bars = base + L::BARS;
+  const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
+  const uint32_t cring = lut + kLutBytes;
+  const uint32_t low = (base + 1023u) & ~1023u;
+  const uint32_t g1 = L::G1 <= lut - low ? low : cring + L::CODES;
+  // byte o of the epilogue buffers
+  auto egap = [lut](uint32_t o) { return lut + ((o >> 7) << 8) + 128u + (o & 127u); };
+  const uint32_t xring = g1 + L::S_X, scring = g1 + L::S_SC, rawring = g1 + L::S_RAW;
+  const uint32_t sus = g1 + L::S_SU, bars = g1 + L::S_BAR;
+  const uint32_t end = base + L::extent(base);
   uint64_t *full = reinterpret_cast<uint64_t *>(gbase + bars);
-  uint64_t *empty = full + kMaxSlots;
-  uint64_t *efull = empty + kMaxSlots;
+  uint64_t *sfull = full + kMaxSlots;
+  uint64_t *empty = sfull + kMaxSlots;
+  uint64_t *rfull = empty + kMaxSlots;   // raw constants by TMA
+  uint64_t *efull = rfull + kMaxSlots;
   uint64_t *eempty = efull + 2;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + bars + L::BARBYTES);
   int *epi_cmd = reinterpret_cast<int *>(gbase + bars + L::BARBYTES + 4);
 
-  if (L::END > dyn_smem_size()) {   // the host sized this; never expected
-    if (threadIdx.x == 0) set_status(P.status, 7 /* QLORA_ERR_CUDA */);
+  if (end > base + dyn_smem_size()) {   // the host sized this; never expected
+    if (threadIdx.x == 0) set_status(Pk.h.status, 7 /* QLORA_ERR_CUDA */);
     return;
   }
 
-  // ---- init: the level table, zero activation rows beyond M, barriers ------
   {
-    // 16-byte stores: four lanes' copies of one entry at a time
-    for (int i = threadIdx.x; i < 2048; i += kSmThreads) {
-      const int e = i >> 3, q4 = i & 7;
-      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(kLambda, c_levels[e >> 4])));
-      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(kLambda, c_levels[e & 15])));
-      const uint32_t v = lo | (hi << 16);
-      *reinterpret_cast<uint4 *>(gbase + lut + e * 256 + q4 * 16) = make_uint4(v, v, v, v);
+    const uint4 *src = reinterpret_cast<const uint4 *>(&Pk.h);
+    uint4 *dst = reinterpret_cast<uint4 *>(&s_head);
+    for (int i = threadIdx.x; i < static_cast<int>(sizeof(SmHead) / 16); i += kSmThreads) dst[i] = src[i];
+  }
+  if (warp == kProducerWarp) {   // the descriptors of this launch's copies
+    const int cnt = Pk.h.count;
+    if (lane < cnt) prefetch_tensormap(&Pk.tm_codes[lane]);
+    if (lane >= 16 && lane - 16 < cnt) prefetch_tensormap(&Pk.tm_x[lane - 16]);
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);    // the producer's arrival with the copies' bytes
+      mbar_init(&sfull[i], kScaleWarps);
+      mbar_init(&empty[i], kConsumerWarps);
+      mbar_init(&rfull[i], 1);
     }
-    if (threadIdx.x == 0) {
-      for (int i = 0; i < NS; ++i) {
-        mbar_init(&full[i], 1 + 32);   // the producer's expect_tx and its lanes' cp.async arrivals
-        mbar_init(&empty[i], kConsumerWarps);
-      }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&efull[i], kConsumerWarps);
-        mbar_init(&eempty[i], kEpiWarps);
-      }
-      *abort_flag = 0;
-      fence_mbarrier_init();
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&efull[i], kConsumerWarps);
+      mbar_init(&eempty[i], kEpiWarps);
     }
+    *abort_flag = 0;
+    fence_mbarrier_init();
   }
   __syncthreads();
+  if (P.pdl) grid_dep_launch();
 
   const int64_t U = P.w_units, G = gridDim.x;
   const int64_t ub = static_cast<int64_t>(blockIdx.x) * U / G, ue = static_cast<int64_t>(blockIdx.x + 1) * U / G;
+
+  // ---- producer pieces ------------------------------------------------------
+  const int sw = warp - kScaleWarp0;   // a scale warp's half of the tile rows
+  // Raw constants of a chunk by cp.async into raw slot rs (one commit group):
+  // for rows lane, lane + 32, ... the chunk's 8 q8 bytes and the second-level
+  // constants of its first and last block.
+  auto issue_raw = [&](const Chunk &k, int rs) {
+    const SmProblem &q = P.p[k.p];
+    const uint32_t sq = rawring + rs * L::RAWSLOT, sd = sq + L::RAWQ8;
+    const int last = (k.kbA + C < q.kblocks ? k.kbA + C : q.kblocks) - 1;
+    const int64_t ngroups = (static_cast<int64_t>(q.N) * q.kblocks + kGroup - 1) / kGroup;
+    const uintptr_t a8 = reinterpret_cast<uintptr_t>(q.scale8);
+    const bool fast8 = (q.kblocks & 7) == 0 && (a8 & 7) == 0;
+    const bool fast4 = (q.kblocks & 3) == 0 && (a8 & 3) == 0;
+#pragma unroll
+    for (int it = 2 * sw; it < 2 * sw + 2; ++it) {
+      const int row = it * 32 + lane;
+      const int64_t n = static_cast<int64_t>(k.tile) * kSmTileRows + row;
+      const uint32_t dq = sq + row * 16 + (k.kbA & 15), dd = sd + row * 8;
+      if (n < q.N) {
+        const int64_t bi = n * q.kblocks + k.kbA;
+        if (fast8) {
+          cp_async_8(dq, q.scale8 + bi);
+        } else if (fast4) {
+          cp_async_4(dq, q.scale8 + bi, 4);
+          cp_async_4(dq + 4, q.scale8 + bi + 4, k.kbA + 4 < q.kblocks ? 4 : 0);
+        } else {   // rows not 4-byte aligned: plain loads (ordered by the wait before use)
+          uint32_t lo = 0, hi = 0;
+          for (int i = 0; i < 8; ++i)
+            if (k.kbA + i < q.kblocks) {
+              const uint32_t v = static_cast<uint32_t>(__ldg(q.scale8 + bi + i));
+              if (i < 4) lo |= v << (8 * i); else hi |= v << (8 * (i - 4));
+            }
+          *reinterpret_cast<uint2 *>(gbase + dq) = make_uint2(lo, hi);
+        }
+        const int64_t ga = bi >> 8, gb = (n * q.kblocks + last) >> 8;
+        cp_async_4(dd, q.scale2 + ga, 4);
+        cp_async_4(dd + 4, q.scale2 + (gb < ngroups ? gb : ga), 4);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // Codes (two 128-row boxes of four blocks) and activations of a chunk into
+  // ring slot `slot`, counted on full[slot]; one thread.
+  auto issue_tma = [&](const Chunk &k, int slot, int chunk_idx) {
+    const SmProblem &q = P.p[k.p];
+    const int nblk = (k.kbA + C < q.kblocks ? k.kbA + C : q.kblocks) - k.kbA;
+    const uint32_t cdst = cring + slot * kCodeSlot, xdst = xring + slot * L::XSLOT;
+    const uint32_t xbytes = (P.x3d ? C : nblk) * L::XBOX;   // a 3-D box counts its zero-filled blocks too
+    mbar_arrive_expect_tx(&full[slot], (nblk > 4 ? 2u : 1u) * (kSmTileRows * 128u) + xbytes);
+    // codes are read once per launch: they should not push the activations,
+    // adapters and partial sums out of L2
+    const uint64_t pol = l2_evict_first_policy();
+    tma_load_2d_hint(gbase + cdst, &Pk.tm_codes[k.p], &full[slot], k.kbA * 32, k.tile * kSmTileRows, pol);
+    if (nblk > 4)
+      tma_load_2d_hint(gbase + cdst + kSmTileRows * 128u, &Pk.tm_codes[k.p], &full[slot], k.kbA * 32 + 128,
+                       k.tile * kSmTileRows, pol);
+    if (chunk_idx == 0 && P.pdl) grid_dep_wait();   // activations may come from the preceding launch
+    if (P.x3d)
+      tma_load_3d(gbase + xdst, &Pk.tm_x[k.p], &full[slot], 0, 0, k.kbA);
+    else
+      for (int b = 0; b < nblk; ++b)
+        tma_load_2d(gbase + xdst + b * L::XBOX, &Pk.tm_x[k.p], &full[slot], (k.kbA + b) * 64, 0);
+  };
+  // Raw constants of a chunk by TMA into raw slot `slot`, counted on
+  // rfull[slot]: the 16-byte column of q8 holding the chunk's 8 blocks for
+  // 128 rows, and 256 second-level constants from the (4-aligned) group of
+  // the tile's first row; one thread.
+  auto issue_raw_tma = [&](const Chunk &k, int slot) {
+    const SmProblem &q = P.p[k.p];
+    const uint32_t sq = rawring + slot * L::RAWSLOT;
+    const int64_t bi0 = static_cast<int64_t>(k.tile) * kSmTileRows * q.kblocks + k.kbA;
+    mbar_arrive_expect_tx(&rfull[slot], L::RAWSLOT);
+    tma_load_2d(gbase + sq, &Pk.tm_q8[k.p], &rfull[slot], k.kbA & ~15, k.tile * kSmTileRows);
+    tma_load_2d(gbase + sq + L::RAWQ8, &Pk.tm_s2[k.p], &rfull[slot], static_cast<int32_t>((bi0 >> 8) & ~int64_t{3}), 0);
+  };
+  // Block scales of a chunk from its raw constants: s = q8 * (d / lambda),
+  // stored [block][row group][g][h] with h = 2 t + hh for weight row
+  // 32 rg + 16 t + 2 g + hh (the rows of a consumer lane); then one arrival
+  // on sfull[slot].
+  auto publish_scales = [&](const Chunk &k, int slot) {
+    const SmProblem &q = P.p[k.p];
+    const uint32_t sq = rawring + slot * L::RAWSLOT, sd = sq + L::RAWQ8;
+    const float *s2w = reinterpret_cast<const float *>(gbase + sd);
+    float *scs = reinterpret_cast<float *>(gbase + scring + slot * L::SCSLOT);
+    const int nblk = (k.kbA + C < q.kblocks ? k.kbA + C : q.kblocks) - k.kbA;
+    const int64_t bi0 = static_cast<int64_t>(k.tile) * kSmTileRows * q.kblocks + k.kbA;
+    const int64_t gw = (bi0 >> 8) & ~int64_t{3};   // first constant of the TMA window
+#pragma unroll
+    for (int it = 2 * sw; it < 2 * sw + 2; ++it) {
+      const int row = it * 32 + lane;
+      const int rgi = row >> 5, wi = row & 31, gi = (wi & 15) >> 1, hi = 2 * (wi >> 4) + (wi & 1);
+      const uint2 q8 = *reinterpret_cast<const uint2 *>(gbase + sq + row * 16 + (k.kbA & 15));
+      const int64_t bi = bi0 + static_cast<int64_t>(row) * q.kblocks;
+      float dA, dB;
+      if (P.rawtma) {
+        dA = s2w[(bi >> 8) - gw];
+        dB = s2w[((bi + nblk - 1) >> 8) - gw];
+      } else {
+        const uint2 dw = *reinterpret_cast<const uint2 *>(gbase + sd + row * 8);
+        dA = __uint_as_float(dw.x);
+        dB = __uint_as_float(dw.y);
+      }
+      const int bnd = 256 - static_cast<int>(bi & 255);
+      const float da = __fmul_rn(dA, kInvLambda), db = __fmul_rn(dB, kInvLambda);
+#pragma unroll
+      for (int i = 0; i < C; ++i) {
+        const uint32_t b = ((i < 4 ? q8.x : q8.y) >> (8 * (i & 3))) & 0xFFu;
+        scs[((i * 4 + rgi) * 8 + gi) * 4 + hi] = static_cast<float>(b) * (i < bnd ? da : db);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sfull[slot]);
+  };
 
   if (warp < kConsumerWarps) {
     // ======================= consumers =======================
     // Warp (rg, slice) owns tile rows 32 rg .. 32 rg + 31 (two 16-row MMA tiles)
     // and the chunk's blocks of parity `slice`.
+    // ---- the level table: entry e (a code byte) at lut + 256 e + 4 lane holds
+    // (bf16(lambda level[e >> 4]), bf16(lambda level[e & 15])) for every lane;
+    // 16-byte stores of four lanes' copies at a time
+    for (int i = threadIdx.x; i < 2048; i += kConsumerWarps * 32) {
+      const int e = i >> 3, q4 = i & 7;
+      const uint32_t v = static_cast<uint32_t>(P.lvl[e >> 4]) | (static_cast<uint32_t>(P.lvl[e & 15]) << 16);
+      *reinterpret_cast<uint4 *>(gbase + lut + e * 256 + q4 * 16) = make_uint4(v, v, v, v);
+    }
+    named_barrier(kTableBar, kConsumerWarps * 32);
+
     const int rg = warp & 3, slice = warp >> 2;
-    const uint32_t lreg = static_cast<uint32_t>(lane * 4);
+    const uint32_t lreg = (lut & 0xFFFF0000u) | static_cast<uint32_t>(lane * 4);
     // code bytes of MMA row g (weight row 2g of a 16-row tile) and row g + 8
     // (weight row 2g + 1): row r of a 128-byte swizzled box holds 16-byte
-    // chunk j at 16 (j ^ (r & 7)); this lane reads 8 bytes at byte 8c of block b
-    const uint32_t hc = static_cast<uint32_t>(c >> 1), sub = static_cast<uint32_t>(8 * (c & 1));
-    uint32_t rbase[2][2], rxor[2][2];
+    // chunk j at 16 (j ^ (r & 7)); this lane reads 8 bytes at byte 8c of a
+    // block. Rows 2g + hh of the two tiles are 2048 bytes apart and share r & 7.
+    const uint32_t hc = static_cast<uint32_t>(c >> 1);
+    // this lane's K 16c .. 16c + 15 of a block are 16-byte chunks 2c and
+    // 2c + 1 of its token's 128-byte row, swizzled by the row's low 3 bits (g)
+    const uint32_t xo0 = static_cast<uint32_t>(((2 * c) ^ g) * 16), xo1 = static_cast<uint32_t>(((2 * c + 1) ^ g) * 16);
+    uint32_t rbase[2], rxor[2];
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t r = static_cast<uint32_t>(32 * rg + 16 * t + 2 * g + hh);
-        rbase[t][hh] = r * 128u + sub;
-        rxor[t][hh] = r & 7u;
-      }
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t r = static_cast<uint32_t>(32 * rg + 2 * g + hh);
+      rbase[hh] = r * 128u + static_cast<uint32_t>(8 * (c & 1));
+      rxor[hh] = r & 7u;
+    }
     float acc[2][NT][4];
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int u = 0; u < NT; ++u) acc[t][u][0] = acc[t][u][1] = acc[t][u][2] = acc[t][u][3] = 0.f;
 
+    Walk wk;
+    walk_init(wk, ub, ue);
+    Chunk cur;
     int chunk_idx = 0, seg_idx = 0;
-    bool ok = true;
-    auto process = [&](const Chunk &cur) {
+    while (walk_next<C>(P, wk, cur)) {
       const int slot = chunk_idx % NS;
-      if (!bar_wait(&full[slot], (chunk_idx / NS) & 1, abort_flag, P.status)) {
-        ok = false;
-        return;
-      }
+      // waits give the same answer on every lane: the MMAs below need the whole warp
+      const uint32_t par = (chunk_idx / NS) & 1;
+      if (!__all_sync(0xffffffffu, bar_wait(&full[slot], par, abort_flag, P.status) &&
+                                       bar_wait(&sfull[slot], par, abort_flag, P.status)))
+        break;
       const uint32_t cs = cring + slot * kCodeSlot;
-      const uint32_t xs = xring + slot * L::XSLOT + g * 512 + 32 * c;
+      const uint32_t xs = xring + slot * L::XSLOT + g * 128;
+      const uint32_t sc = scring + slot * L::SCSLOT + ((rg * 8 + g) * 4) * 4;
       const int f = cur.kb_s + (((cur.kb_s & 1) != slice) ? 1 : 0);
       const int nown = f < cur.kb_e ? (cur.kb_e - f + 1) / 2 : 0;
-      // block scales fp32(q8 * d) / lambda of this lane's four rows (2g, 2g + 1
-      // of both tiles) for its own blocks of the chunk; block i of a row uses
-      // the first block's second-level constant up to the 256-block group
-      // boundary and the last block's after it
-      const SmProblem &q = P.p[cur.p];
-      float sc[D][4];
+      // one 64-K block (chunk-local index kbl) of the warp's 32 rows
+      auto block = [&](int kbl) {
+        const uint32_t half = cs + static_cast<uint32_t>(kbl >> 2) * (kSmTileRows * 128u);
+        const uint32_t jj = 2u * static_cast<uint32_t>(kbl & 3) + hc;
+        uint2 w[2][2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int row = 32 * rg + 16 * (j >> 1) + 2 * g + (j & 1);
-        const uint32_t sq = sring + slot * L::SSLOT + row * 8;
-        uint2 q8w, dw;
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(q8w.x), "=r"(q8w.y) : "r"(sq));
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(dw.x), "=r"(dw.y) : "r"(sq + kSmTileRows * 8));
-        const int64_t bi = (static_cast<int64_t>(cur.tile) * kSmTileRows + row) * q.kblocks + cur.kbA;
-        const int bnd = 256 - static_cast<int>(bi & 255);
-        const float da = __fmul_rn(__uint_as_float(dw.x), kInvLambda), db = __fmul_rn(__uint_as_float(dw.y), kInvLambda);
-#pragma unroll
-        for (int s = 0; s < D; ++s) {
-          const int kbl = f + 2 * s - cur.kbA;
-          const uint32_t q8v = prmt(q8w.x, q8w.y, 0x4440u | static_cast<uint32_t>(kbl & 7)) & 0xFFu;
-          sc[s][j] = static_cast<float>(q8v) * (kbl < bnd ? da : db);
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t a = half + rbase[hh] + 16u * (jj ^ rxor[hh]);
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0][hh].x), "=r"(w[0][hh].y) : "r"(a));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2+2048];" : "=r"(w[1][hh].x), "=r"(w[1][hh].y) : "r"(a));
         }
-      }
+        // activations: token 8u + g is row 8u + g of the block's swizzled box
+        uint4 x[NT][2];
+        const uint32_t xb = xs + static_cast<uint32_t>(kbl) * L::XBOX;
 #pragma unroll
-      for (int s = 0; s < D; ++s) {
-        if (s < nown) {
-          const int kbl = f + 2 * s - cur.kbA;
-          const uint32_t half = cs + static_cast<uint32_t>(kbl >> 2) * (kSmTileRows * 128u);
-          const uint32_t jj = 2u * static_cast<uint32_t>(kbl & 3) + hc;
-          uint2 w[2][2];
+        for (int u = 0; u < NT; ++u) {
+          x[u][0] = lds_u128(xb + u * 1024 + xo0);
+          x[u][1] = lds_u128(xb + u * 1024 + xo1);
+        }
+        float4 sv;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(sv.x), "=f"(sv.y), "=f"(sv.z), "=f"(sv.w)
+                     : "r"(sc + kbl * (kSmTileRows * 4)));
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t) {
+          // the four k-steps of the block in two independent chains (steps
+          // 0, 2 and 1, 3), added before the block scale
+          float tmp[2][NT][4];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const uint32_t a = half + rbase[t][hh] + 16u * (jj ^ rxor[t][hh]);
-              asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[t][hh].x), "=r"(w[t][hh].y) : "r"(a));
-            }
-          uint4 x[NT][2];
-          const uint32_t xb = xs + static_cast<uint32_t>(kbl >> 2) * L::XBOX + (kbl & 3) * 128;
-#pragma unroll
-          for (int u = 0; u < NT; ++u) {
-            x[u][0] = lds_u128(xb + u * 8 * 512);
-            x[u][1] = lds_u128(xb + u * 8 * 512 + 16);
-          }
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            // the four k-steps of the block in two independent chains (steps
-            // 0, 2 and 1, 3), added before the block scale
-            float tmp[2][NT][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t wa = (i >> 1) ? w[t][0].y : w[t][0].x, wb = (i >> 1) ? w[t][1].y : w[t][1].x;
-              const uint32_t sel0 = 0x7604u | ((static_cast<uint32_t>(2 * i) & 3u) << 4);
-              const uint32_t sel1 = 0x7604u | ((static_cast<uint32_t>(2 * i + 1) & 3u) << 4);
-              const uint32_t a0 = lds_u32(lut + prmt(wa, lreg, sel0));   // MMA row g,     K 4i, 4i+1 of the lane's 16
-              const uint32_t a1 = lds_u32(lut + prmt(wb, lreg, sel0));   // MMA row g + 8
-              const uint32_t a2 = lds_u32(lut + prmt(wa, lreg, sel1));   // MMA row g,     K 4i+2, 4i+3
-              const uint32_t a3 = lds_u32(lut + prmt(wb, lreg, sel1));   // MMA row g + 8
-#pragma unroll
-              for (int u = 0; u < NT; ++u) {
-                const uint32_t b0 = (i == 0) ? x[u][0].x : (i == 1) ? x[u][0].z : (i == 2) ? x[u][1].x : x[u][1].z;
-                const uint32_t b1 = (i == 0) ? x[u][0].y : (i == 1) ? x[u][0].w : (i == 2) ? x[u][1].y : x[u][1].w;
-                if (i < 2)
-                  mma_zero(tmp[i][u], a0, a1, a2, a3, b0, b1);
-                else
-                  mma_acc(tmp[i & 1][u], a0, a1, a2, a3, b0, b1);
-              }
-            }
-            const float s_lo = sc[s][2 * t], s_hi = sc[s][2 * t + 1];
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t wa = (i >> 1) ? w[t][0].y : w[t][0].x, wb = (i >> 1) ? w[t][1].y : w[t][1].x;
+            const uint32_t sel0 = 0x7604u | ((static_cast<uint32_t>(2 * i) & 3u) << 4);
+            const uint32_t sel1 = 0x7604u | ((static_cast<uint32_t>(2 * i + 1) & 3u) << 4);
+            const uint32_t a0 = lds_u32(prmt(wa, lreg, sel0));   // MMA row g,     K 4i, 4i+1 of the lane's 16
+            const uint32_t a1 = lds_u32(prmt(wb, lreg, sel0));   // MMA row g + 8
+            const uint32_t a2 = lds_u32(prmt(wa, lreg, sel1));   // MMA row g,     K 4i+2, 4i+3
+            const uint32_t a3 = lds_u32(prmt(wb, lreg, sel1));   // MMA row g + 8
 #pragma unroll
             for (int u = 0; u < NT; ++u) {
-              acc[t][u][0] = fmaf(tmp[0][u][0] + tmp[1][u][0], s_lo, acc[t][u][0]);
-              acc[t][u][1] = fmaf(tmp[0][u][1] + tmp[1][u][1], s_lo, acc[t][u][1]);
-              acc[t][u][2] = fmaf(tmp[0][u][2] + tmp[1][u][2], s_hi, acc[t][u][2]);
-              acc[t][u][3] = fmaf(tmp[0][u][3] + tmp[1][u][3], s_hi, acc[t][u][3]);
+              const uint32_t b0 = (i == 0) ? x[u][0].x : (i == 1) ? x[u][0].z : (i == 2) ? x[u][1].x : x[u][1].z;
+              const uint32_t b1 = (i == 0) ? x[u][0].y : (i == 1) ? x[u][0].w : (i == 2) ? x[u][1].y : x[u][1].w;
+              if (i < 2)
+                mma_zero(tmp[i][u], a0, a1, a2, a3, b0, b1);
+              else
+                mma_acc(tmp[i & 1][u], a0, a1, a2, a3, b0, b1);
             }
           }
+          const float s_lo = t == 0 ? sv.x : sv.z, s_hi = t == 0 ? sv.y : sv.w;
+#pragma unroll
+          for (int u = 0; u < NT; ++u) {
+            acc[t][u][0] = fmaf(tmp[0][u][0] + tmp[1][u][0], s_lo, acc[t][u][0]);
+            acc[t][u][1] = fmaf(tmp[0][u][1] + tmp[1][u][1], s_lo, acc[t][u][1]);
+            acc[t][u][2] = fmaf(tmp[0][u][2] + tmp[1][u][2], s_hi, acc[t][u][2]);
+            acc[t][u][3] = fmaf(tmp[0][u][3] + tmp[1][u][3], s_hi, acc[t][u][3]);
+          }
         }
+      };
+      if (nown == D) {   // a whole chunk: no branches between the blocks
+#pragma unroll
+        for (int s = 0; s < D; ++s) block(f + 2 * s - cur.kbA);
+      } else {
+#pragma unroll
+        for (int s = 0; s < D; ++s)
+          if (s < nown) block(f + 2 * s - cur.kbA);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
 
       if (cur.last) {   // hand the segment's sums to the epilogue warps
         const int eb = seg_idx & 1;
-        if (!bar_wait(&eempty[eb], ((seg_idx >> 1) & 1) ^ 1, abort_flag, P.status)) {
-          ok = false;
-          return;
-        }
-        float *dst = reinterpret_cast<float *>(gbase + ebuf + eb * L::EBUF) + slice * kSmTileRows * L::EROW;
+        if (!__all_sync(0xffffffffu, bar_wait(&eempty[eb], ((seg_idx >> 1) & 1) ^ 1, abort_flag, P.status))) break;
+        const uint32_t ob = eb * L::EBUF + slice * kSmTileRows * L::EROW * 4;
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int u = 0; u < NT; ++u) {
-            const int row = 32 * rg + 16 * t + 2 * g;   // weight rows of MMA rows g and g + 8
-            *reinterpret_cast<float2 *>(dst + row * L::EROW + 8 * u + 2 * c) = make_float2(acc[t][u][0], acc[t][u][1]);
-            *reinterpret_cast<float2 *>(dst + (row + 1) * L::EROW + 8 * u + 2 * c) =
-                make_float2(acc[t][u][2], acc[t][u][3]);
+            const uint32_t row = 32 * rg + 16 * t + 2 * g;   // weight rows of MMA rows g and g + 8
+            const uint32_t o = ob + (row * L::EROW + 8 * u + 2 * c) * 4;
+            *reinterpret_cast<float2 *>(gbase + egap(o)) = make_float2(acc[t][u][0], acc[t][u][1]);
+            *reinterpret_cast<float2 *>(gbase + egap(o + L::EROW * 4)) = make_float2(acc[t][u][2], acc[t][u][3]);
             acc[t][u][0] = acc[t][u][1] = acc[t][u][2] = acc[t][u][3] = 0.f;
           }
         __syncwarp();
@@ -496,93 +655,100 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
         ++seg_idx;
       }
       ++chunk_idx;
-    };
-
-    Walk wk;
-    walk_init(wk, ub, ue);
-    Chunk cur;
-    while (ok && walk_next<C>(P, wk, cur)) process(cur);
+    }
   } else if (warp == kProducerWarp) {
     // ======================= producer =======================
-    // Per chunk: two TMA boxes of codes and two of activations (lane 0), and
-    // each lane's share of the block constants by cp.async: for rows lane,
-    // lane + 32, ... the 8 constants of the chunk and the second-level
-    // constants of the chunk's first and last block.
-    Walk wk;
-    walk_init(wk, ub, ue);
-    Chunk k;
-    int chunk_idx = 0;
-    while (walk_next<C>(P, wk, k)) {
-      const int slot = chunk_idx % NS;
-      if (!bar_wait(&empty[slot], ((chunk_idx / NS) & 1) ^ 1, abort_flag, P.status, 32)) break;
-      {
-        const SmProblem &q = P.p[k.p];
-        const uint32_t sq = sring + slot * L::SSLOT, sd = sq + kSmTileRows * 8;
-        const int last = (k.kbA + C < q.kblocks ? k.kbA + C : q.kblocks) - 1;
-        const int64_t ngroups = (static_cast<int64_t>(q.N) * q.kblocks + kGroup - 1) / kGroup;
-        // 8- or 4-byte copies where every row's 8 constants start aligned
-        const uintptr_t a8 = reinterpret_cast<uintptr_t>(q.scale8);
-        const bool fast8 = (q.kblocks & 7) == 0 && (a8 & 7) == 0;
-        const bool fast4 = (q.kblocks & 3) == 0 && (a8 & 3) == 0;
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int row = it * 32 + lane;
-          const int64_t n = static_cast<int64_t>(k.tile) * kSmTileRows + row;
-          const uint32_t dq = sq + row * 8, dd = sd + row * 8;
-          if (n < q.N) {
-            const int64_t bi = n * q.kblocks + k.kbA;
-            if (fast8) {
-              cp_async_8(dq, q.scale8 + bi);
-            } else if (fast4) {
-              cp_async_4(dq, q.scale8 + bi, 4);
-              cp_async_4(dq + 4, q.scale8 + bi + 4, k.kbA + 4 < q.kblocks ? 4 : 0);
-            } else {   // rows not 4-byte aligned: plain loads
-              uint32_t lo = 0, hi = 0;
-              for (int i = 0; i < 8; ++i)
-                if (k.kbA + i < q.kblocks) {
-                  const uint32_t v = static_cast<uint32_t>(__ldg(q.scale8 + bi + i));
-                  if (i < 4) lo |= v << (8 * i); else hi |= v << (8 * (i - 4));
-                }
-              *reinterpret_cast<uint2 *>(gbase + dq) = make_uint2(lo, hi);
-            }
-            const int64_t ga = bi >> 8, gb = (n * q.kblocks + last) >> 8;
-            cp_async_4(dd, q.scale2 + ga, 4);
-            cp_async_4(dd + 4, q.scale2 + (gb < ngroups ? gb : ga), 4);
+    // One thread: per chunk, wait for its slot (from the NS-th chunk on) and
+    // request its copies.
+    if (lane == 0) {
+      Walk pwk;
+      walk_init(pwk, ub, ue);
+      Chunk k;
+      int n = 0;   // chunks whose copies were requested
+      while (walk_next<C>(P, pwk, k)) {
+        const int slot = n % NS;
+        if (n >= NS && !bar_wait(&empty[slot], ((n / NS) & 1) ^ 1, abort_flag, P.status, 32)) break;
+        issue_tma(k, slot, n);
+        ++n;
+      }
+      // do not leave while copies into this CTA's shared memory may be in flight
+      if (*abort_flag) {
+        for (int i = n - 1; i >= 0 && i >= n - NS; --i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[i % NS], (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
           }
         }
-        if (fast4) {
-          cp_async_arrive(&full[slot]);
-        } else {   // plain stores above: complete the copies, then a releasing arrival
-          asm volatile("cp.async.wait_all;" ::: "memory");
-          mbar_arrive(&full[slot]);
-        }
       }
-      if (lane == 0) {
-        const SmProblem &q = P.p[k.p];
-        const int nblk = (k.kbA + C < q.kblocks ? k.kbA + C : q.kblocks) - k.kbA;
-        const uint32_t cdst = cring + slot * kCodeSlot, xdst = xring + slot * L::XSLOT;
-        uint32_t tx = kSmTileRows * 128u + L::XBOX;
-        if (chunk_idx == 0 && P.pdl) grid_dep_wait();   // activations may come from the preceding launch
-        tma_load_2d(gbase + cdst, &P.tm_codes[k.p], &full[slot], k.kbA * 32, k.tile * kSmTileRows);
-        tma_load_2d(gbase + xdst, &P.tm_x[k.p], &full[slot], k.kbA * 64, 0);
-        if (nblk > 4) {
-          tma_load_2d(gbase + cdst + kSmTileRows * 128u, &P.tm_codes[k.p], &full[slot], k.kbA * 32 + 128,
-                      k.tile * kSmTileRows);
-          tma_load_2d(gbase + xdst + L::XBOX, &P.tm_x[k.p], &full[slot], k.kbA * 64 + 256, 0);
-          tx += kSmTileRows * 128u + L::XBOX;
-        }
-        mbar_arrive_expect_tx(&full[slot], tx);
-      }
-      __syncwarp();
-      ++chunk_idx;
     }
-    // do not leave while copies into this CTA's shared memory may be in flight
-    if (*abort_flag && chunk_idx > 0) {
-      for (int i = chunk_idx - 1; i >= 0 && i >= chunk_idx - NS; --i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&full[i % NS], (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+  } else if (warp < kScaleWarp0 + kScaleWarps) {
+    // ======================= block scales =======================
+    // The raw constants of chunk c are requested NS chunks ahead (when chunk
+    // c - NS has been published, into the raw slot it used); per chunk: wait
+    // for its slot, then for its raw constants, then publish its scales.
+    Walk rwk, swk;
+    walk_init(rwk, ub, ue);
+    walk_init(swk, ub, ue);
+    Chunk kr, k;
+    int nraw = 0, n = 0;
+    const bool issuer = sw == 0 && lane == 0;   // requests the raw constants of both warps
+    if (P.rawtma) {
+      if (issuer)
+        for (; nraw < NS && walk_next<C>(P, rwk, kr); ++nraw) issue_raw_tma(kr, nraw);
+      while (walk_next<C>(P, swk, k)) {
+        const int slot = n % NS;
+        if (n >= NS &&
+            !__all_sync(0xffffffffu, bar_wait(&empty[slot], ((n / NS) & 1) ^ 1, abort_flag, P.status, 32)))
+          break;
+        if (!__all_sync(0xffffffffu, bar_wait(&rfull[slot], (n / NS) & 1, abort_flag, P.status))) break;
+        publish_scales(k, slot);
+        // the slot's raw constants were read by both warps: the second warp
+        // arrives on sfull only after reading them
+        bool ok = true;
+        if (issuer && walk_next<C>(P, rwk, kr)) {
+          ok = bar_wait(&sfull[slot], (n / NS) & 1, abort_flag, P.status);
+          if (ok) {
+            issue_raw_tma(kr, slot);
+            ++nraw;
+          }
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
+        ++n;
+      }
+      // do not leave while copies into this CTA's shared memory may be in flight
+      if (issuer && *abort_flag) {
+        for (int i = nraw - 1; i >= 0 && i >= nraw - NS; --i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&rfull[i % NS], (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
         }
       }
+    } else {
+    for (int i = 0; i < NS; ++i) {
+      if (!walk_next<C>(P, rwk, kr)) break;
+      issue_raw(kr, i);
+      ++nraw;
+    }
+    while (walk_next<C>(P, swk, k)) {
+      const int slot = n % NS;
+      if (n >= NS &&
+          !__all_sync(0xffffffffu, bar_wait(&empty[slot], ((n / NS) & 1) ^ 1, abort_flag, P.status, 32)))
+        break;
+      const int pend = nraw - n - 1;   // raw groups that may stay in flight
+      if (pend >= 2)
+        asm volatile("cp.async.wait_group 2;" ::: "memory");
+      else if (pend == 1)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncwarp();
+      publish_scales(k, slot);
+      if (walk_next<C>(P, rwk, kr)) {
+        issue_raw(kr, slot);
+        ++nraw;
+      }
+      ++n;
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
   } else {
     // ======================= epilogue =======================
@@ -593,7 +759,8 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
     // ---- pieces of X A^T: 128 K each, every load issued before the MMAs ----
     // Inside each 64-K block the K order is permuted as in the weight path: lane
     // (g, c) holds K 16c .. 16c + 15 of a row, so its fragments are two 16-byte
-    // loads per row and block.
+    // loads per row and block. The piece that completes a linear's set adds all
+    // of them in order and publishes sU = bf16(s X A^T).
     for (int64_t qi = static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew; qi < P.u_units;
          qi += static_cast<int64_t>(gridDim.x) * kEpiWarps) {
       int p = 0;
@@ -658,13 +825,53 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
             *reinterpret_cast<float2 *>(up + (j + 8) * MP + t) = make_float2(d[jt][u][2], d[jt][u][3]);
           }
       __syncwarp();
+      unsigned long long old = 0;
       if (lane == 0) {
         __threadfence();   // after the warp barrier: covers the whole warp's partial sums
-        atomicAdd(&P.ucnt[p], 1ull);
+        old = atomicAdd(&P.ucnt[p], 1ull);
+      }
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old + 1 == static_cast<unsigned long long>(q.uchunks)) {
+        // the last piece: U = the pieces summed in piece order (16 loads in
+        // flight per lane), sU = bf16(s U), then the linear's ready flag
+        __threadfence();
+        const int cols = 16 * r16 * MP / 4;   // float4 columns of one piece
+        for (int col = lane; col < cols; col += 32) {
+          const float4 *src4 = reinterpret_cast<const float4 *>(q.upart) + col;
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+          int cc = 0;
+          for (; cc + 16 <= q.uchunks; cc += 16) {
+            float4 v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __ldcg(src4 + static_cast<int64_t>(cc + e) * cols);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              a.x += v[e].x; a.y += v[e].y; a.z += v[e].z; a.w += v[e].w;
+            }
+          }
+          for (; cc < q.uchunks; ++cc) {
+            const float4 v = __ldcg(src4 + static_cast<int64_t>(cc) * cols);
+            a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+          }
+          const int j = (4 * col) / MP, t0 = (4 * col) % MP;
+          const float uv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (j < q.r && t0 + e < P.M)
+              q.sU[static_cast<int64_t>(t0 + e) * q.r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(q.s * uv[e]));
+        }
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          st_release_gpu_u64(&P.flags[G + p], P.epoch);
+        }
       }
     }
 
     // ---- finished segments ----
+    // Before waiting for a segment that finishes a tile, the epilogue already
+    // fetches that linear's sU (once per CTA and linear) and the tile's rows of
+    // B, so only the sums and the stores remain after the wait.
     float *su_s = reinterpret_cast<float *>(gbase + sus);
     int su_p = -1;   // the linear whose sU su_s holds
     Walk wk;
@@ -674,14 +881,48 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
     const int64_t self = blockIdx.x;
     while (walk_next<C>(P, wk, k)) {
       if (!k.last) continue;
+      const SmProblem &q = P.p[k.p];
+      const int64_t n = static_cast<int64_t>(k.tile) * kSmTileRows + et;
+      const bool tile_first = k.seg_lo == 0, tile_last = k.seg_hi == q.kblocks;
+      // rows of B held in registers across the wait: all 64 ranks for 8
+      // tokens, the first 32 for 16 (the rest is loaded after it)
+      constexpr int BPRE = NT == 2 ? 4 : 8;
+      uint4 bpre[BPRE];
+      const uint4 *brow = reinterpret_cast<const uint4 *>(q.B + n * q.r);
+      if (tile_first) {
+        if (k.p != su_p) {
+          // the barrier also ends every read of su_s for the previous linear;
+          // every path through a segment passes a barrier after reading epi_cmd[1]
+          if (q.sU_in == nullptr && et == 0)
+            epi_cmd[1] = wait_word(&P.flags[G + k.p], P.epoch, abort_flag, P.status) ? 1 : 0;
+          named_barrier(kEpiBar, kEpiWarps * 32);
+          if (q.sU_in == nullptr && epi_cmd[1] == 0) break;
+          const uint16_t *sUp = q.sU_in ? q.sU_in : q.sU;
+          for (int i = et; i < P.M * q.r; i += kEpiWarps * 32) {
+            const int t = i / q.r, j = i % q.r;
+            su_s[t * 64 + j] = __uint_as_float(static_cast<uint32_t>(__ldcg(sUp + i)) << 16);
+          }
+          su_p = k.p;
+        }
+        if (n < q.N) {
+#pragma unroll
+          for (int j8 = 0; j8 < BPRE; ++j8)
+            if (j8 < q.r / 8) bpre[j8] = __ldg(brow + j8);
+        }
+      }
       const int eb = seg_idx & 1;
-      if (!bar_wait(&efull[eb], (seg_idx >> 1) & 1, abort_flag, P.status, 64)) break;
-      const float *src = reinterpret_cast<const float *>(gbase + ebuf + eb * L::EBUF);
+      // one thread waits and the barrier hands its answer to the others, so
+      // all 128 leave together on a timeout (every later path passes a
+      // barrier before epi_cmd[2] is written again)
+      if (et == 0) epi_cmd[2] = bar_wait(&efull[eb], (seg_idx >> 1) & 1, abort_flag, P.status, 64) ? 1 : 0;
+      named_barrier(kEpiBar, kEpiWarps * 32);
+      if (epi_cmd[2] == 0) break;
       float sum[MP];
 #pragma unroll
       for (int t = 0; t < MP; t += 4) {
-        const float4 a = *reinterpret_cast<const float4 *>(src + et * L::EROW + t);
-        const float4 b = *reinterpret_cast<const float4 *>(src + (kSmTileRows + et) * L::EROW + t);
+        const uint32_t o = eb * L::EBUF + (et * L::EROW + t) * 4;
+        const float4 a = *reinterpret_cast<const float4 *>(gbase + egap(o));
+        const float4 b = *reinterpret_cast<const float4 *>(gbase + egap(o + kSmTileRows * L::EROW * 4));
         sum[t] = a.x + b.x;
         sum[t + 1] = a.y + b.y;
         sum[t + 2] = a.z + b.z;
@@ -691,9 +932,6 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
       if (lane == 0) mbar_arrive(&eempty[eb]);
       ++seg_idx;
 
-      const SmProblem &q = P.p[k.p];
-      const int64_t n = static_cast<int64_t>(k.tile) * kSmTileRows + et;
-      const bool tile_first = k.seg_lo == 0, tile_last = k.seg_hi == q.kblocks;
       if (!tile_first) {
         // a later contributor: publish the partial for the CTA holding the tile's first block
         float *slot = P.slots + self * (MP * kSmTileRows);
@@ -732,99 +970,36 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
         named_barrier(kEpiBar, kEpiWarps * 32);
         if (et == 0)
           for (int bb = static_cast<int>(self) + 1; bb <= b1; ++bb) P.flags[bb] = 0;
+      } else {
+        named_barrier(kEpiBar, kEpiWarps * 32);   // su_s is complete
       }
       // finish the tile: the LoRA term in fp32, then Y in bf16
-      if (k.p != su_p) {   // sU of this linear, once per CTA
-        if (q.sU_in != nullptr) {
-          for (int i = et; i < P.M * q.r; i += kEpiWarps * 32) {
-            const int t = i / q.r, j = i % q.r;
-            su_s[t * 64 + j] = __uint_as_float(static_cast<uint32_t>(__ldg(q.sU_in + i)) << 16);
-          }
-        } else {
-          // wait for every piece of X A^T, then add them in a fixed order:
-          // thread (part, col) sums pieces part, part + nsplit, ... of float4
-          // column col; the parts are then added in order
-          if (et == 0)
-            epi_cmd[0] = wait_word(reinterpret_cast<const uint64_t *>(&P.ucnt[k.p]),
-                                   static_cast<uint64_t>(q.uchunks), abort_flag, P.status) ? 1 : 0;
-          named_barrier(kEpiBar, kEpiWarps * 32);
-          if (epi_cmd[0] == 0) break;
-          const int r16 = (q.r + 15) / 16;
-          const int cols = 16 * r16 * MP / 4;                 // float4 columns of one piece
-          const int nsplit = cols >= 128 ? 1 : 128 / cols;    // 1, 2 or 4 (cols is 32, 64, 128 ...)
-          float4 *red4 = reinterpret_cast<float4 *>(gbase + reds);
-          for (int col0 = 0; col0 < cols; col0 += 128 / nsplit) {
-            const int col = col0 + et % (128 / nsplit), part = et / (128 / nsplit);
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (col < cols) {
-              const float4 *src4 = reinterpret_cast<const float4 *>(q.upart) + col;
-              int cc = part;
-              for (; cc + 3 * nsplit < q.uchunks; cc += 4 * nsplit) {
-                const float4 v0 = __ldcg(src4 + static_cast<int64_t>(cc) * cols);
-                const float4 v1 = __ldcg(src4 + static_cast<int64_t>(cc + nsplit) * cols);
-                const float4 v2 = __ldcg(src4 + static_cast<int64_t>(cc + 2 * nsplit) * cols);
-                const float4 v3 = __ldcg(src4 + static_cast<int64_t>(cc + 3 * nsplit) * cols);
-                a.x += v0.x; a.y += v0.y; a.z += v0.z; a.w += v0.w;
-                a.x += v1.x; a.y += v1.y; a.z += v1.z; a.w += v1.w;
-                a.x += v2.x; a.y += v2.y; a.z += v2.z; a.w += v2.w;
-                a.x += v3.x; a.y += v3.y; a.z += v3.z; a.w += v3.w;
-              }
-              for (; cc < q.uchunks; cc += nsplit) {
-                const float4 v = __ldcg(src4 + static_cast<int64_t>(cc) * cols);
-                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
-              }
-            }
-            red4[et] = a;
-            named_barrier(kEpiBar, kEpiWarps * 32);
-            if (part == 0 && col < cols) {
-              float4 t4 = red4[et];
-              for (int pp = 1; pp < nsplit; ++pp) {
-                const float4 v = red4[et + pp * (128 / nsplit)];
-                t4.x += v.x; t4.y += v.y; t4.z += v.z; t4.w += v.w;
-              }
-              // column col holds U[j][t .. t + 3] with j = 4 col / MP, t = 4 col % MP
-              const int j = (4 * col) / MP, t0 = (4 * col) % MP;
-              const float uv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int t = t0 + e;
-                if (j < q.r && t < P.M) {
-                  const __nv_bfloat16 b = __float2bfloat16_rn(q.s * uv[e]);
-                  su_s[t * 64 + j] = __bfloat162float(b);
-                  if (k.tile == 0) q.sU[static_cast<int64_t>(t) * q.r + j] = __bfloat16_as_ushort(b);
-                }
-              }
-            }
-            named_barrier(kEpiBar, kEpiWarps * 32);
-          }
-        }
-        su_p = k.p;
-      }
-      named_barrier(kEpiBar, kEpiWarps * 32);
       if (n < q.N) {
         float y[MP];
 #pragma unroll
         for (int t = 0; t < MP; ++t) y[t] = sum[t];
-        const uint4 *brow = reinterpret_cast<const uint4 *>(q.B + n * q.r);
-        for (int j8 = 0; j8 < q.r / 8; ++j8) {
-          const uint4 bv = __ldg(brow + j8);
-          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            const float bj = __uint_as_float((h & 1) ? (bw[h >> 1] & 0xFFFF0000u) : (bw[h >> 1] << 16));
+        for (int j8 = 0; j8 < 8; ++j8) {
+          if (j8 < q.r / 8) {
+            const uint4 bv = j8 < BPRE ? bpre[j8 < BPRE ? j8 : 0] : __ldg(brow + j8);
+            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-            for (int t = 0; t < MP; ++t) y[t] = fmaf(su_s[t * 64 + 8 * j8 + h], bj, y[t]);
+            for (int h = 0; h < 8; ++h) {
+              const float bj = __uint_as_float((h & 1) ? (bw[h >> 1] & 0xFFFF0000u) : (bw[h >> 1] << 16));
+#pragma unroll
+              for (int t = 0; t < MP; ++t) y[t] = fmaf(su_s[t * 64 + 8 * j8 + h], bj, y[t]);
+            }
           }
         }
 #pragma unroll
         for (int t = 0; t < MP; ++t)
           if (t < P.M) q.Y[static_cast<int64_t>(t) * q.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[t]));
       }
-      named_barrier(kEpiBar, kEpiWarps * 32);
       if (q.sU_in == nullptr && et == 0) {
         if (atomicAdd(&P.ucons[k.p], 1ull) + 1 == static_cast<unsigned long long>(q.tiles)) {   // the last user
           atomicExch(&P.ucnt[k.p], 0ull);
           atomicExch(&P.ucons[k.p], 0ull);
+          P.flags[G + k.p] = 0;
         }
       }
     }
@@ -841,6 +1016,16 @@ uint64_t next_epoch() {
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
+// bf16(lambda * level[i]): the fp32 product rounded to nearest even (the
+// levels and lambda are finite and far from the bf16 range limits).
+uint16_t lambda_level_bf16(int i) {
+  static const float levels[16] = QLORA_NF4_LEVELS;
+  const float v = kLambda * levels[i];
+  uint32_t b;
+  std::memcpy(&b, &v, 4);
+  return static_cast<uint16_t>((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+}
+
 struct SmWsLayout {
   size_t flags, slots, total;
   size_t upart[kSmMaxProblems], su[kSmMaxProblems];
@@ -851,8 +1036,8 @@ SmWsLayout sm_ws_layout(const SmallProblem *pr, int count, int64_t M) {
   const size_t G = static_cast<size_t>(device_sm_count());
   const int MP = M <= 8 ? 8 : 16;
   size_t off = 0;
-  w.flags = off;
-  off += up256(G * 8);
+  w.flags = off;   // [G] published partials, then [kSmMaxProblems] sU ready
+  off += up256((G + kSmMaxProblems) * 8);
   w.slots = off;
   off += up256(G * MP * kSmTileRows * 4);
   for (int i = 0; i < count; ++i) {
@@ -894,8 +1079,12 @@ cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *w
     const SmWsLayout w = sm_ws_layout(q, n, M);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     SmParams P{};
-    P.count = n;
-    P.M = static_cast<int32_t>(M);
+    SmHead &H = P.h;
+    H.count = n;
+    H.M = static_cast<int32_t>(M);
+    for (int i = 0; i < 16; ++i) H.lvl[i] = lambda_level_bf16(i);
+    const uint32_t mp = M > 8 ? 16 : 8;
+    bool all3d = true;
     int64_t wu = 0;
     int32_t uu = 0;
     for (int i = 0; i < n; ++i) {
@@ -903,11 +1092,14 @@ cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *w
                      static_cast<uint64_t>(q[i].N), static_cast<uint64_t>(q[i].K / 2), 128, kSmTileRows,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-      if (!encode_2d(&P.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q[i].X, static_cast<uint64_t>(q[i].K),
-                     static_cast<uint64_t>(M), static_cast<uint64_t>(q[i].K) * 2, 256, M > 8 ? 16 : 8,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-      SmProblem &p = P.p[i];
+      // activations as [K/64 blocks][M tokens][64]: one box holds a chunk's
+      // 8 blocks for MP tokens, each token row 128 bytes, swizzled
+      const uint64_t xd[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(q[i].K / kBlock)};
+      const uint64_t xs[2] = {static_cast<uint64_t>(q[i].K) * 2, 128};
+      const uint32_t xb[3] = {64, mp, static_cast<uint32_t>(kChunkBlocks)};
+      all3d = all3d && encode_3d(&P.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q[i].X, xd, xs, xb,
+                                 CU_TENSOR_MAP_SWIZZLE_128B);
+      SmProblem &p = H.p[i];
       p.codes = q[i].codes;
       p.scale8 = q[i].scale8;
       p.scale2 = q[i].scale2;
@@ -936,15 +1128,38 @@ cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *w
         p.sU = nullptr;
       }
     }
-    P.w_units = wu;
-    P.u_units = uu;
-    P.epoch = next_epoch();
-    P.flags = reinterpret_cast<uint64_t *>(wsb + w.flags);
-    P.ucnt = static_cast<unsigned long long *>(counters);
-    P.ucons = P.ucnt + kSmMaxProblems;
-    P.slots = reinterpret_cast<float *>(wsb + w.slots);
-    P.status = status;
-    P.pdl = pdl ? 1 : 0;
+    if (!all3d)   // else one 2-D box per block, for every linear of the launch
+      for (int i = 0; i < n; ++i)
+        if (!encode_2d(&P.tm_x[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q[i].X, static_cast<uint64_t>(q[i].K),
+                       static_cast<uint64_t>(M), static_cast<uint64_t>(q[i].K) * 2, 64, mp,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+          return cudaErrorInvalidValue;
+    H.x3d = all3d ? 1 : 0;
+    // raw constants by TMA when every linear allows it: q8 rows a multiple
+    // of 16 bytes, a window of 256 second-level constants covering a chunk's
+    // 128 rows (at most 480 blocks a row), 16-byte aligned arrays
+    bool rawtma = true;
+    for (int i = 0; i < n && rawtma; ++i) {
+      const int64_t kb = q[i].K / kBlock;
+      const uint64_t ngroups = static_cast<uint64_t>((q[i].N * kb + kGroup - 1) / kGroup);
+      rawtma = kb % 16 == 0 && kb <= 480 && reinterpret_cast<uintptr_t>(q[i].scale8) % 16 == 0 &&
+               reinterpret_cast<uintptr_t>(q[i].scale2) % 16 == 0 &&
+               encode_2d(&P.tm_q8[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, q[i].scale8, static_cast<uint64_t>(kb),
+                         static_cast<uint64_t>(q[i].N), static_cast<uint64_t>(kb), 16, kSmTileRows,
+                         CU_TENSOR_MAP_SWIZZLE_NONE) &&
+               encode_2d(&P.tm_s2[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, q[i].scale2, ngroups, 1,
+                         (ngroups * 4 + 15) / 16 * 16, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    H.rawtma = rawtma ? 1 : 0;
+    H.w_units = wu;
+    H.u_units = uu;
+    H.epoch = next_epoch();
+    H.flags = reinterpret_cast<uint64_t *>(wsb + w.flags);
+    H.ucnt = static_cast<unsigned long long *>(counters);
+    H.ucons = H.ucnt + kSmMaxProblems;
+    H.slots = reinterpret_cast<float *>(wsb + w.slots);
+    H.status = status;
+    H.pdl = pdl ? 1 : 0;
 
     const int sms = device_sm_count();
     const int grid = static_cast<int>(wu < sms ? wu : sms);
