@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);    // the producer's arrival with the copies' bytes
+      mbar_init(&full[i], 1);   // the producer's arrival with the copies' bytes
       mbar_init(&sfull[i], kScaleWarps);
       mbar_init(&empty[i], kConsumerWarps);
       mbar_init(&rfull[i], 1);
@@ -825,16 +825,15 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
             *reinterpret_cast<float2 *>(up + (j + 8) * MP + t) = make_float2(d[jt][u][2], d[jt][u][3]);
           }
       __syncwarp();
+      // the count releases the warp's partial sums (ordered before lane 0's add
+      // by the warp barrier) and acquires the other pieces' for the last one
       unsigned long long old = 0;
-      if (lane == 0) {
-        __threadfence();   // after the warp barrier: covers the whole warp's partial sums
-        old = atomicAdd(&P.ucnt[p], 1ull);
-      }
+      if (lane == 0) old = atom_add_acq_rel_gpu(&P.ucnt[p], 1ull);
       old = __shfl_sync(0xffffffffu, old, 0);
+      __syncwarp();
       if (old + 1 == static_cast<unsigned long long>(q.uchunks)) {
         // the last piece: U = the pieces summed in piece order (16 loads in
         // flight per lane), sU = bf16(s U), then the linear's ready flag
-        __threadfence();
         const int cols = 16 * r16 * MP / 4;   // float4 columns of one piece
         for (int col = lane; col < cols; col += 32) {
           const float4 *src4 = reinterpret_cast<const float4 *>(q.upart) + col;
@@ -860,11 +859,8 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
             if (j < q.r && t0 + e < P.M)
               q.sU[static_cast<int64_t>(t0 + e) * q.r + j] = __bfloat16_as_ushort(__float2bfloat16_rn(q.s * uv[e]));
         }
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          st_release_gpu_u64(&P.flags[G + p], P.epoch);
-        }
+        __syncwarp();   // the release below covers the whole warp's sU stores
+        if (lane == 0) st_release_gpu_u64(&P.flags[G + p], P.epoch);
       }
     }
 
@@ -941,10 +937,7 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
         // the barrier orders every thread's stores before thread 0's release,
         // which is cumulative: the flag publishes all of them at GPU scope
         named_barrier(kEpiBar, kEpiWarps * 32);
-        if (et == 0) {
-          __threadfence();
-          st_release_gpu_u64(&P.flags[self], P.epoch);
-        }
+        if (et == 0) st_release_gpu_u64(&P.flags[self], P.epoch);
         continue;
       }
       if (!tile_last) {
@@ -961,7 +954,23 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
         const bool ok = epi_cmd[0] != 0;
         named_barrier(kEpiBar, kEpiWarps * 32);
         if (!ok) break;
-        for (int bb = static_cast<int>(self) + 1; bb <= b1; ++bb) {
+        // four contributors' partials are loaded before they are added (in CTA order)
+        constexpr int CB = MP == 8 ? 4 : 2;
+        int bb = static_cast<int>(self) + 1;
+        for (; bb + CB - 1 <= b1; bb += CB) {
+          float v[CB][MP];
+#pragma unroll
+          for (int i = 0; i < CB; ++i) {
+            const float *slot = P.slots + static_cast<int64_t>(bb + i) * (MP * kSmTileRows);
+#pragma unroll
+            for (int t = 0; t < MP; ++t) v[i][t] = t < P.M ? __ldcg(slot + t * kSmTileRows + et) : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < CB; ++i)
+#pragma unroll
+            for (int t = 0; t < MP; ++t) sum[t] += v[i][t];
+        }
+        for (; bb <= b1; ++bb) {
           const float *slot = P.slots + static_cast<int64_t>(bb) * (MP * kSmTileRows);
 #pragma unroll
           for (int t = 0; t < MP; ++t)
@@ -983,11 +992,22 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
           if (j8 < q.r / 8) {
             const uint4 bv = j8 < BPRE ? bpre[j8 < BPRE ? j8 : 0] : __ldg(brow + j8);
             const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+            float bj[8];
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-              const float bj = __uint_as_float((h & 1) ? (bw[h >> 1] & 0xFFFF0000u) : (bw[h >> 1] << 16));
+            for (int h = 0; h < 8; ++h)
+              bj[h] = __uint_as_float((h & 1) ? (bw[h >> 1] & 0xFFFF0000u) : (bw[h >> 1] << 16));
 #pragma unroll
-              for (int t = 0; t < MP; ++t) y[t] = fmaf(su_s[t * 64 + 8 * j8 + h], bj, y[t]);
+            for (int t = 0; t < MP; ++t) {   // sU[t][8 j8 .. 8 j8 + 7] in two 16-byte loads (same address for all threads)
+              const float4 sa = *reinterpret_cast<const float4 *>(su_s + t * 64 + 8 * j8);
+              const float4 sb = *reinterpret_cast<const float4 *>(su_s + t * 64 + 8 * j8 + 4);
+              y[t] = fmaf(sa.x, bj[0], y[t]);
+              y[t] = fmaf(sa.y, bj[1], y[t]);
+              y[t] = fmaf(sa.z, bj[2], y[t]);
+              y[t] = fmaf(sa.w, bj[3], y[t]);
+              y[t] = fmaf(sb.x, bj[4], y[t]);
+              y[t] = fmaf(sb.y, bj[5], y[t]);
+              y[t] = fmaf(sb.z, bj[6], y[t]);
+              y[t] = fmaf(sb.w, bj[7], y[t]);
             }
           }
         }

@@ -253,6 +253,15 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Atomic add at GPU scope that releases this thread's earlier writes (and
+// those ordered before it by a barrier) and acquires the writes released by
+// earlier adds to the same word; returns the old value.
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_gpu(unsigned long long *p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
 // Flag publication between CTAs of one grid (global memory, GPU scope).
 __device__ __forceinline__ void st_release_gpu_u64(uint64_t *p, uint64_t v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
