@@ -49,7 +49,103 @@ def parse_args():
     p.add_argument("--oracle-configs", action="store_true",
                    help="time the CPU oracle on every workload (host only) and print one JSON line")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--kernel-case", choices=sorted(KERNEL_CASES),
+                   help="run one kernel family on its profiling workload (3 calls, then one more) and exit; "
+                        "for ncu -k <kernel> -s 3 -c 1")
     return p.parse_args()
+
+
+def _kc_setup():
+    import torch
+    import bit_nf4_quantized_dequant_b200 as q
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    bf = lambda *shape, sc=1.0: (torch.randn(*shape, generator=g, device="cuda") * sc).bfloat16()
+    w = lambda n, k: torch.randn(n, k, generator=g, device="cuda") * 0.02
+    return torch, q, bf, w
+
+
+def _kc_dequant():
+    torch, q, bf, w = _kc_setup()
+    m = q.nf4_quantize(w(8192, 8192))
+    o = torch.empty(8192, 8192, dtype=torch.bfloat16, device="cuda")
+    return lambda: q.nf4_dequantize(m, out=o)
+
+
+def _kc_quantize():
+    torch, q, bf, w = _kc_setup()
+    W, m = w(8192, 8192), q.NF4Matrix.empty(8192, 8192, "cuda")
+    return lambda: q.nf4_quantize(W, out=m)
+
+
+def _kc_merge():
+    torch, q, bf, w = _kc_setup()
+    N, K, r = 4096, 14336, 16
+    m, A, B = q.nf4_quantize(w(N, K)), bf(r, K, sc=0.01), bf(N, r, sc=0.01)
+    o = torch.empty(N, K, dtype=torch.bfloat16, device="cuda")
+    return lambda: q.nf4_merge(m, A, B, 2.0, out=o)
+
+
+def _kc_linear():
+    torch, q, bf, w = _kc_setup()
+    M, N, K, r = 2048, 4096, 4096, 16
+    m, X, A, B, dY = q.nf4_quantize(w(N, K)), bf(M, K), bf(r, K, sc=0.01), bf(N, r, sc=0.01), bf(M, N)
+    ws = torch.zeros(q.linear_workspace(M, N, K, r), dtype=torch.uint8, device="cuda")
+
+    def step():
+        Y, sU = q.linear_fwd(m, X, A, B, 2.0, ws=ws)
+        q.linear_bwd(m, X, A, B, 2.0, dY, sU=sU, ws=ws)
+    return step
+
+
+def _kc_swiglu():
+    torch, q, bf, w = _kc_setup()
+    M, H, F, r = 4096, 4096, 11008, 16
+    qgu = q.nf4_quantize(q.swiglu_interleave(w(F, H), w(F, H)))
+    X, Bgu = bf(M, H), q.swiglu_pack_b(bf(F, r, sc=0.01), bf(F, r, sc=0.01))
+    sU, dH = bf(M, 2 * r, sc=0.1), bf(M, F)
+
+    def step():
+        q.swiglu_fwd(qgu, X, Bgu, sU)
+        q.swiglu_bwd(qgu, X, Bgu, sU, dH)
+    return step
+
+
+def _kc_decode():
+    # one grouped few-token launch of eight 8B linears (193 MB of codes, more
+    # than L2), L2 flushed before each call
+    torch, q, bf, w = _kc_setup()
+    M, r = 8, 16
+    probs, X = [], {}
+    for (N, K) in [(14336, 4096)] * 4 + [(4096, 14336)] * 2 + [(4096, 4096)] * 2:
+        if K not in X:
+            X[K] = bf(M, K)
+        probs.append(q.LinearProblem(q.nf4_quantize(w(N, K)), X[K], bf(r, K, sc=0.06), bf(N, r, sc=0.01), 2.0,
+                                     torch.empty(M, N, dtype=torch.bfloat16, device="cuda"),
+                                     torch.empty(M, r, dtype=torch.bfloat16, device="cuda")))
+    ws = torch.zeros(q.linear_fwd_group_workspace(probs, M), dtype=torch.uint8, device="cuda")
+    arr = q._binding._problem_array(probs)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        flush.zero_()
+        q.linear_fwd_group(probs, ws=ws, arr=arr)
+    return step
+
+
+KERNEL_CASES = {"dequant": _kc_dequant, "quantize": _kc_quantize, "merge": _kc_merge, "linear": _kc_linear,
+                "swiglu": _kc_swiglu, "decode": _kc_decode}
+
+
+def run_kernel_case(name):
+    import torch
+    from bit_nf4_quantized_dequant_b200 import _build
+    _build.build()
+    f = KERNEL_CASES[name]()
+    for _ in range(4):
+        f()
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": name, "calls": 4}))
 
 
 def load_peaks():
@@ -873,6 +969,8 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 def main():
     args = parse_args()
+    if args.kernel_case:
+        return run_kernel_case(args.kernel_case)
     if args.impl == "reference":
         run_reference(args)
         return

@@ -59,11 +59,49 @@ Thresholds thresholds_for(const float (&L)[16]) {
   return th;
 }
 
-__device__ __forceinline__ uint32_t nearest_code(float n, const Thresholds &th) {
-  uint32_t code = 0;
-#pragma unroll
-  for (int i = 0; i < 15; ++i) code += n >= th.t[i] ? 1u : 0u;
-  return code;
+// The same count with one comparison: [-1, 1] is cut into 129 cells of
+// width 1/64, cell j = floor(64 n + 64 + off); cand[j] thresholds lie below
+// the cell and at most one, t[j], inside it (+inf if none), so
+// code = cand[j] + (n >= t[j]). `off` keeps every threshold at least 1/1000
+// of a cell away from the cell edges, so the rounding of 64 n + 64 + off can
+// move n to a neighbouring cell only where both cells give the same count.
+struct CellTable {
+  float t[129];
+  int32_t cand[129];
+  float off64;   // 64 + off
+};
+
+bool cell_table_for(const Thresholds &th, CellTable *ct) {
+  static const double offs[] = {0.5, 0.25, 0.75, 0.125, 0.375, 0.625, 0.875, 0.0625, 0.3125, 0.5625, 0.8125};
+  for (const double off : offs) {
+    bool ok = true;
+    for (int i = 0; i < 15 && ok; ++i) {
+      const double x = 64.0 * th.t[i] + 64.0 + off, f = x - std::floor(x);
+      ok = f > 1e-3 && f < 1.0 - 1e-3;
+    }
+    for (int j = 0; j <= 128 && ok; ++j) {
+      const double lo = (j - 64 - off) / 64.0, hi = lo + 1.0 / 64.0;
+      int cand = 0, inside = 0;
+      float t = std::numeric_limits<float>::infinity();
+      for (int i = 0; i < 15; ++i) {
+        if (th.t[i] < lo) ++cand;
+        else if (th.t[i] < hi) { ++inside; t = th.t[i]; }
+      }
+      ok = inside <= 1;
+      ct->t[j] = t;
+      ct->cand[j] = cand;
+    }
+    if (ok) {
+      ct->off64 = static_cast<float>(64.0 + off);
+      return true;
+    }
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint32_t cell_code(float n, const float *ts, const int32_t *cs, float off64) {
+  const int j = __float2int_rd(fmaf(n, 64.f, off64));   // n in [-1, 1]: j in [0, 128]
+  return static_cast<uint32_t>(cs[j]) + (n >= ts[j] ? 1u : 0u);
 }
 
 // One CTA per group of 256 blocks. A warp load covers two consecutive blocks
@@ -78,8 +116,15 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
                                                            uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scale8,
                                                            float *__restrict__ scale2,
-                                                           int32_t *status, const Thresholds th) {
+                                                           int32_t *status, const CellTable ct) {
   __shared__ float c1s[kGroup];
+  __shared__ float cts[129];
+  __shared__ int32_t ccs[129];
+  for (int i = threadIdx.x; i < 129; i += blockDim.x) {
+    cts[i] = ct.t[i];
+    ccs[i] = ct.cand[i];
+  }
+  __syncthreads();
   __shared__ float red[8];
   __shared__ float mu_s;
   const int64_t g = blockIdx.x;
@@ -111,10 +156,10 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float *__restri
       constexpr uint32_t kZero = BOOK == kBookInt4 ? 8u : 7u;   // index of the exact zero level
       uint32_t e0 = kZero, e1 = kZero, e2 = kZero, e3 = kZero;
       if (m > 0.f) {
-        e0 = nearest_code(__fdiv_rn(v[u].x, m), th);
-        e1 = nearest_code(__fdiv_rn(v[u].y, m), th);
-        e2 = nearest_code(__fdiv_rn(v[u].z, m), th);
-        e3 = nearest_code(__fdiv_rn(v[u].w, m), th);
+        e0 = cell_code(__fdiv_rn(v[u].x, m), cts, ccs, ct.off64);
+        e1 = cell_code(__fdiv_rn(v[u].y, m), cts, ccs, ct.off64);
+        e2 = cell_code(__fdiv_rn(v[u].z, m), cts, ccs, ct.off64);
+        e3 = cell_code(__fdiv_rn(v[u].w, m), cts, ccs, ct.off64);
       }
       if (i < nblk) {
         // bytes 2hl, 2hl+1 of the block: (e0 << 4 | e1), (e2 << 4 | e3)
@@ -229,20 +274,19 @@ cudaError_t launch_quantize(const float *W, int64_t rows, int64_t cols, uint8_t 
     if (e != cudaSuccess) return e;
   }
   const unsigned grid = static_cast<unsigned>(ng);
-  static const Thresholds th_nf4 = [] {
-    const float L[16] = QLORA_NF4_LEVELS;
-    return thresholds_for(L);
+  static CellTable ct_nf4, ct_int4;
+  static const bool ct_ok = [] {
+    const float Ln[16] = QLORA_NF4_LEVELS;
+    const float Li[16] = QLORA_INT4_LEVELS;
+    return cell_table_for(thresholds_for(Ln), &ct_nf4) && cell_table_for(thresholds_for(Li), &ct_int4);
   }();
-  static const Thresholds th_int4 = [] {
-    const float L[16] = QLORA_INT4_LEVELS;
-    return thresholds_for(L);
-  }();
+  if (!ct_ok) return cudaErrorInvalidValue;   // no offset separates the thresholds from the cell edges (never expected)
   if (dq == kDqFp8)
-    nf4_quantize_kernel<kBookNf4, kDqFp8><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_nf4);
+    nf4_quantize_kernel<kBookNf4, kDqFp8><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, ct_nf4);
   else if (book == kBookInt4)
-    nf4_quantize_kernel<kBookInt4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_int4);
+    nf4_quantize_kernel<kBookInt4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, ct_int4);
   else
-    nf4_quantize_kernel<kBookNf4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, th_nf4);
+    nf4_quantize_kernel<kBookNf4, kDqLinear><<<grid, 256, 0, s>>>(W, nb, codes, scale8, scale2, dev_status, ct_nf4);
   return cudaGetLastError();
 }
 

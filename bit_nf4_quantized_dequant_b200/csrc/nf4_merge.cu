@@ -179,21 +179,26 @@ cudaError_t launch_merge_t(const uint8_t *codes, const uint8_t *scale8, const fl
                            int64_t K, const uint16_t *Al, const uint16_t *Bl, int r, float s, void *out,
                            cudaStream_t st) {
   const int64_t strips = (K + kCols - 1) / kCols;
-  // enough CTAs for about four per SM, each a band of rows (multiple of 16)
-  const int64_t want = 4 * static_cast<int64_t>(device_sm_count());
-  int64_t bands = (want + strips - 1) / strips;
-  if (bands > N / 16) bands = N / 16;
-  if (bands < 1) bands = 1;
-  int64_t rows_per = (N + bands - 1) / bands;
-  rows_per = (rows_per + 15) / 16 * 16;
-  bands = (N + rows_per - 1) / rows_per;
-  const dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(bands));
-  const int rp = static_cast<int>(rows_per);
   const size_t dyn = kF32Out ? 0 : static_cast<size_t>(kMergeWarps) * 16 * 512;
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kMergeWarps * 32, dyn, st>>>(codes, scale8, scale2, N, K, Al, Bl, r, s, out, rp);
+    // one wave: as many (strip, band) CTAs as are resident at once, each a
+    // band of rows (a multiple of 16); a second partial wave would leave most
+    // SMs idle for its whole length
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kMergeWarps * 32, dyn);
+    if (e != cudaSuccess) return e;
+    const int64_t resident = static_cast<int64_t>(per_sm > 0 ? per_sm : 1) * device_sm_count();
+    int64_t bands = resident / strips;
+    if (bands > N / 16) bands = N / 16;
+    if (bands < 1) bands = 1;
+    int64_t rows_per = (N + bands - 1) / bands;
+    rows_per = (rows_per + 15) / 16 * 16;
+    bands = (N + rows_per - 1) / rows_per;
+    const dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(bands));
+    kernel<<<grid, kMergeWarps * 32, dyn, st>>>(codes, scale8, scale2, N, K, Al, Bl, r, s, out,
+                                                static_cast<int>(rows_per));
     return cudaGetLastError();
   };
   switch ((r + 15) / 16) {

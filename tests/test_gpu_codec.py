@@ -171,3 +171,54 @@ def test_fp8_and_linear_second_levels_err_alike(lib):
     e_lin = torch.sqrt(torch.mean((lin - W) ** 2)).item()
     e_f8 = torch.sqrt(torch.mean((f8 - W) ** 2)).item()
     assert abs(e_f8 - e_lin) < 0.03 * e_lin
+
+
+def _boundary_weights(levels, seed):
+    """Blocks whose quotients w / c1 fall within a few float32 steps of every
+    decision point between adjacent levels, and of every multiple of 1/128
+    (where an implementation may switch between internal search ranges), for
+    block maxima of very different magnitudes. Element 0 of each block is +-c1
+    so that c1 is the block's absmax."""
+    rng = np.random.default_rng(seed)
+    lv = np.asarray(levels, dtype=np.float64)
+    points = [0.5 * (lv[i] + lv[i + 1]) for i in range(15)] + [k / 128.0 for k in range(-127, 128)]
+    vals = []
+    for p in points:
+        x = np.float32(p)
+        for k in range(-4, 5):
+            y = x
+            for _ in range(abs(k)):
+                y = np.nextafter(y, np.float32(np.inf if k > 0 else -np.inf))
+            vals.append(y)
+    vals = np.clip(np.array(vals, dtype=np.float32), -1, 1)
+    rows = []
+    for c1 in (1.0, 0.0371, 3.0517578e-5, 7.5e3, float(rng.uniform(0.01, 0.2))):
+        c1 = np.float32(c1)
+        q = (vals.astype(np.float64) * np.float64(c1)).astype(np.float32)   # w near c1 * point
+        pad = (-q.size) % 63
+        q = np.concatenate([q, np.zeros(pad, np.float32)]).reshape(-1, 63)
+        blk = np.concatenate([np.full((q.shape[0], 1), c1, np.float32), q], axis=1)
+        blk[::2, 0] = -c1
+        rows.append(blk)
+    flat = np.concatenate(rows).reshape(-1)
+    flat = np.concatenate([flat, np.zeros((-flat.size) % 512, np.float32)])
+    return flat.reshape(-1, 512)
+
+
+def test_quantize_codes_at_decision_points(lib):
+    """Codes of quotients a few float32 steps either side of each level
+    midpoint (and of the multiples of 1/128) match the oracle for NF4 and for
+    the int4 comparison codebook ("QLoRA, in depth", "The mechanism in brief":
+    nearest of the 16 levels)."""
+    import torch
+    from oracle import codebooks
+    W = _boundary_weights(onf4.nf4_levels(), 21)
+    q, st = _quantize_gpu(lib, W)
+    assert st == 0
+    codes, s8, s2 = onf4.quantize(W)
+    assert np.array_equal(q.codes.cpu().numpy(), codes)
+    W4 = _boundary_weights(codebooks.int4_levels(), 22)
+    q4 = lib.codec_quantize(torch.from_numpy(W4).cuda(), lib.CODEBOOK_INT4)
+    torch.cuda.synchronize()
+    p4, _, _ = codebooks.quantize_int4(W4)
+    np.testing.assert_array_equal(q4.codes.cpu().numpy(), p4)
