@@ -100,7 +100,9 @@ bool cell_table_for(const Thresholds &th, CellTable *ct) {
 }
 
 __device__ __forceinline__ uint32_t cell_code(float n, const float *ts, const int32_t *cs, float off64) {
-  const int j = __float2int_rd(fmaf(n, 64.f, off64));   // n in [-1, 1]: j in [0, 128]
+  // n in [-1, 1] gives j in [0, 128]; the clamp keeps the quotient of a
+  // non-finite weight (reported through the status) inside the table
+  const int j = min(max(__float2int_rd(fmaf(n, 64.f, off64)), 0), 128);
   return static_cast<uint32_t>(cs[j]) + (n >= ts[j] ? 1u : 0u);
 }
 
