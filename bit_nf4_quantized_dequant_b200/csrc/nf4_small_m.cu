@@ -75,7 +75,7 @@ bool encode_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, co
 
 namespace {
 
-constexpr int kSmMaxProblems = 8;
+constexpr int kSmMaxProblems = 16;                  // linears per launch (the counter page holds 2 x 16 counters)
 constexpr int kSmTileRows = 128;
 constexpr int kConsumerWarps = 8;                    // 4 row groups x 2 K slices
 constexpr int kProducerWarp = 8;                     // the copies of codes and activations
@@ -131,6 +131,7 @@ struct __align__(16) SmHead {
   uint16_t lvl[16];        // bf16(lambda * level[i])
 };
 static_assert(sizeof(SmHead) % 16 == 0, "copied as 16-byte words");
+static_assert(2 * kSmMaxProblems * 8 <= kSmallCounterBytes, "ucnt and ucons fit the counter page");
 
 struct SmParams {
   CUtensorMap tm_codes[kSmMaxProblems];   // codes of each linear as u8 [N][K/2], 128 x 128-byte boxes, swizzled
@@ -312,7 +313,8 @@ struct Layout {
   static constexpr uint32_t S_SC = S_X + NS * XSLOT;
   static constexpr uint32_t S_RAW = S_SC + NS * SCSLOT;
   static constexpr uint32_t S_SU = S_RAW + NS * RAWSLOT;
-  static constexpr uint32_t S_BAR = S_SU + SUBYTES;
+  static constexpr uint32_t S_HEAD = S_SU + SUBYTES;        // the launch's head (parameters)
+  static constexpr uint32_t S_BAR = S_HEAD + static_cast<uint32_t>(sizeof(SmHead));
   static constexpr uint32_t G1 = S_BAR + BARBYTES + 16;
   static constexpr uint32_t CODES = NS * kCodeSlot;
   // bytes used from the start of dynamic shared memory at shared address
@@ -339,8 +341,6 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
   constexpr int NS = L::NS;
   constexpr int D = C / 2;   // own blocks of a consumer warp per chunk
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ SmHead s_head;
-  const SmHead &P = s_head;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -356,6 +356,8 @@ __global__ void __launch_bounds__(kSmThreads, 1) nf4_small_m_kernel(const __grid
   auto egap = [lut](uint32_t o) { return lut + ((o >> 7) << 8) + 128u + (o & 127u); };
   const uint32_t xring = g1 + L::S_X, scring = g1 + L::S_SC, rawring = g1 + L::S_RAW;
   const uint32_t sus = g1 + L::S_SU, bars = g1 + L::S_BAR;
+  SmHead &s_head = *reinterpret_cast<SmHead *>(gbase + g1 + L::S_HEAD);
+  const SmHead &P = s_head;
   const uint32_t end = base + L::extent(base);
   uint64_t *full = reinterpret_cast<uint64_t *>(gbase + bars);
   uint64_t *sfull = full + kMaxSlots;

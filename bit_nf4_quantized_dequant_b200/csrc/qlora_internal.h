@@ -125,7 +125,7 @@ struct SmallProblem {
 // first launch and that every launch leaves zero (nothing else may write them).
 constexpr size_t kSmallCounterBytes = 256;
 size_t small_m_ws_bytes(const SmallProblem *pr, int count, int64_t M);
-// One launch per 8 linears, in order on `st`; with pdl the launch may start
+// One launch per 16 linears, in order on `st`; with pdl the launch may start
 // streaming the weights before the preceding work on the stream has finished.
 cudaError_t launch_small_m(const SmallProblem *pr, int count, int64_t M, void *ws, void *counters, bool pdl,
                            int32_t *status, cudaStream_t st);

@@ -233,7 +233,7 @@ qlora_status_t qlora_linear_bwd(const qlora_nf4_t *W, const uint16_t *X, int64_t
  *   captured call can be replayed); one call at a time may use it. After a
  *   QLORA_ERR_TIMEOUT in dev_status the workspace must be zero-filled (or
  *   replaced) before it is used again.
- * More than 8 problems run as consecutive launches of 8 on `stream`.
+ * More than 16 problems run as consecutive launches of 16 on `stream`.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (M > 16, or a shape qlora_linear_fwd
  * rejects), MISALIGNED, WORKSPACE, CUDA; TIMEOUT in dev_status.
  */
