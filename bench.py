@@ -112,12 +112,14 @@ def _kc_swiglu():
 
 
 def _kc_decode():
-    # one grouped few-token launch of eight 8B linears (193 MB of codes, more
-    # than L2), L2 flushed before each call
+    # one grouped few-token launch of sixteen 8B linears (two layers' q, k, v,
+    # o, gate, up, down, then q and k: 266 MB of codes, more than L2), L2
+    # flushed before each call
     torch, q, bf, w = _kc_setup()
     M, r = 8, 16
     probs, X = [], {}
-    for (N, K) in [(14336, 4096)] * 4 + [(4096, 14336)] * 2 + [(4096, 4096)] * 2:
+    layer = [(4096, 4096), (1024, 4096), (1024, 4096), (4096, 4096), (14336, 4096), (14336, 4096), (4096, 14336)]
+    for (N, K) in layer * 2 + layer[:2]:
         if K not in X:
             X[K] = bf(M, K)
         probs.append(q.LinearProblem(q.nf4_quantize(w(N, K)), X[K], bf(r, K, sc=0.06), bf(N, r, sc=0.01), 2.0,
