@@ -113,7 +113,7 @@ def _kc_swiglu():
 
 def _kc_decode():
     # one grouped few-token launch of sixteen 8B linears (two layers' q, k, v,
-    # o, gate, up, down, then q and k: 266 MB of codes, more than L2), L2
+    # o, gate, up, down, then q and k: 236 MB of codes, more than L2), L2
     # flushed before each call
     torch, q, bf, w = _kc_setup()
     M, r = 8, 16
