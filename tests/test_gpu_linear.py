@@ -206,14 +206,19 @@ def test_stream_k_graph_replays(lib):
     del g
 
 
-# Few-token forwards take the weight-streaming kernel (dequantisation into
-# warp-MMA register fragments, K split over a thread-block cluster).
+# Few-token forwards take the persistent weight-streaming kernel (codes,
+# activations and block constants through a shared-memory ring, warp-level MMAs,
+# tiles split between CTAs). The block constants come by TMA when a row's 8-bit
+# constants are a multiple of 16 bytes and a chunk's second-level constants fit
+# one 256-entry window (at most 480 blocks a row), else by cp.async.
 FEW_TOKEN_CASES = [
     # N, K, M, r
-    (1024, 7168, 5, 16),    # cluster of 8, 14 NF4 blocks per CTA: a ragged last span
-    (512, 4096, 16, 32),    # two token tiles of 8
+    (1024, 7168, 5, 16),    # 112 blocks a row: constants by TMA
+    (512, 4096, 16, 32),    # 16 tokens (two MMA token tiles)
     (2048, 1024, 9, 8),     # second token tile nearly empty
-    (64, 192, 3, 64),       # one row group, three blocks, largest rank
+    (64, 192, 3, 64),       # one tile, three blocks (byte-wise constants), largest rank
+    (256, 32768, 8, 16),    # 512 blocks a row: constants by cp.async; 256 pieces of X A^T
+    (384, 11008, 7, 24),    # 172 blocks a row (not a multiple of 16): cp.async; rank 24
 ]
 
 
