@@ -15,10 +15,12 @@
 //   (32 KB of codes) into a shared-memory ring with two 2-D TMA copies
 //   (128-byte swizzle) and the chunk's activations with two more (token rows
 //   beyond M arrive as zeros), so HBM sees whole 128-byte row segments and no
-//   warp holds loads in flight in its registers. The chunk's 8-bit block
-//   constants and second-level constants arrive in the same ring (cp.async,
-//   completing on the chunk's barrier); the consumer warps form the block
-//   scales of their own rows from there.
+//   warp holds loads in flight in its registers.
+// * Two scale warps bring the chunk's 8-bit block constants and its
+//   second-level constants into a ring of their own (a TMA copy of each, or
+//   cp.async where K does not suit the copy's 16-byte rule), form the fp32
+//   block scales of all 128 rows and publish them in a third ring, laid out
+//   in the order the consumer lanes read them.
 // * Every code byte becomes a bf16 pair with one PRMT and one shared-memory
 //   load: a 256-entry table of (level[hi nibble], level[lo nibble]) pairs,
 //   one copy per lane in that lane's own bank (64 KB, each entry's row of 256
