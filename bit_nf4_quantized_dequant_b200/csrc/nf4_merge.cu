@@ -20,6 +20,8 @@
 // rows padded so that those loads hit 32 distinct banks. bf16 results go
 // through a per-warp shared-memory tile (16-byte chunks XOR-swizzled within
 // each block, conflict-free both ways) and leave as whole 512-byte rows.
+#include <atomic>
+
 #include "qlora_device.cuh"
 
 namespace qlora {
@@ -174,22 +176,53 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 2)
   }
 }
 
+// Resident CTAs per SM of one kernel instantiation, found (with its shared
+// memory limit raised) on the first launch on each device and kept: the
+// query costs microseconds of host time, which a pass over many small
+// matrices would otherwise pay per launch.
+constexpr int kMergeMaxDevices = 64;
+
+template <typename Kernel>
+cudaError_t merge_blocks_per_sm(Kernel kernel, size_t dyn, std::atomic<int> (&cache)[kMergeMaxDevices], int *per_sm) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < kMergeMaxDevices;
+  if (cacheable) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) {
+      *per_sm = v;
+      return cudaSuccess;
+    }
+  }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
+  if (e != cudaSuccess) return e;
+  int n = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kMergeWarps * 32, dyn);
+  if (e != cudaSuccess) return e;
+  if (n < 1) n = 1;
+  if (cacheable) cache[dev].store(n, std::memory_order_relaxed);
+  *per_sm = n;
+  return cudaSuccess;
+}
+
+template <bool kF32Out, int KSTEPS>
+std::atomic<int> g_merge_per_sm[kMergeMaxDevices];
+
 template <bool kF32Out>
 cudaError_t launch_merge_t(const uint8_t *codes, const uint8_t *scale8, const float *scale2, int64_t N,
                            int64_t K, const uint16_t *Al, const uint16_t *Bl, int r, float s, void *out,
                            cudaStream_t st) {
   const int64_t strips = (K + kCols - 1) / kCols;
   const size_t dyn = kF32Out ? 0 : static_cast<size_t>(kMergeWarps) * 16 * 512;
-  auto go = [&](auto kernel) -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn));
-    if (e != cudaSuccess) return e;
+  auto go = [&](auto kernel, std::atomic<int> (&cache)[kMergeMaxDevices]) -> cudaError_t {
     // one wave: as many (strip, band) CTAs as are resident at once, each a
     // band of rows (a multiple of 16); a second partial wave would leave most
     // SMs idle for its whole length
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kMergeWarps * 32, dyn);
+    cudaError_t e = merge_blocks_per_sm(kernel, dyn, cache, &per_sm);
     if (e != cudaSuccess) return e;
-    const int64_t resident = static_cast<int64_t>(per_sm > 0 ? per_sm : 1) * device_sm_count();
+    const int64_t resident = static_cast<int64_t>(per_sm) * device_sm_count();
     int64_t bands = resident / strips;
     if (bands > N / 16) bands = N / 16;
     if (bands < 1) bands = 1;
@@ -202,10 +235,10 @@ cudaError_t launch_merge_t(const uint8_t *codes, const uint8_t *scale8, const fl
     return cudaGetLastError();
   };
   switch ((r + 15) / 16) {
-    case 1: return go(nf4_merge_kernel<kF32Out, 1>);
-    case 2: return go(nf4_merge_kernel<kF32Out, 2>);
-    case 3: return go(nf4_merge_kernel<kF32Out, 3>);
-    case 4: return go(nf4_merge_kernel<kF32Out, 4>);
+    case 1: return go(nf4_merge_kernel<kF32Out, 1>, g_merge_per_sm<kF32Out, 1>);
+    case 2: return go(nf4_merge_kernel<kF32Out, 2>, g_merge_per_sm<kF32Out, 2>);
+    case 3: return go(nf4_merge_kernel<kF32Out, 3>, g_merge_per_sm<kF32Out, 3>);
+    case 4: return go(nf4_merge_kernel<kF32Out, 4>, g_merge_per_sm<kF32Out, 4>);
     default: return cudaErrorInvalidValue;
   }
 }

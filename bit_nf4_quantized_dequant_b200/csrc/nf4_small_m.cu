@@ -51,7 +51,7 @@
 //   publish or finish the tile while the consumers stream on, and add the
 //   LoRA term sU B^T in fp32 before the single bf16 rounding of Y.
 // * sU = bf16(s X A^T) is formed in the same launch: at the start the
-//   epilogue warps of all CTAs split X A^T into 256-K pieces, the last piece
+//   epilogue warps of all CTAs split X A^T into 128-K pieces, the last piece
 //   of a linear to arrive sums them in order and publishes sU, and tiles wait
 //   (bounded) for it before their LoRA term.
 //

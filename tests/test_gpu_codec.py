@@ -177,7 +177,7 @@ def _boundary_weights(levels, seed):
     """Blocks whose quotients w / c1 fall within a few float32 steps of every
     decision point between adjacent levels, and of every multiple of 1/128
     (where an implementation may switch between internal search ranges), for
-    block maxima of very different magnitudes. Element 0 of each block is +-c1
+    block maxima of very different magnitudes, down to subnormal products. Element 0 of each block is +-c1
     so that c1 is the block's absmax."""
     rng = np.random.default_rng(seed)
     lv = np.asarray(levels, dtype=np.float64)
@@ -192,7 +192,10 @@ def _boundary_weights(levels, seed):
             vals.append(y)
     vals = np.clip(np.array(vals, dtype=np.float32), -1, 1)
     rows = []
-    for c1 in (1.0, 0.0371, 3.0517578e-5, 7.5e3, float(rng.uniform(0.01, 0.2))):
+    # maxima either side of 2^-125 and 2^126, where a quotient taken through
+    # the reciprocal of c1 would leave the normal range
+    edges = (2.0 ** -125, 2.0 ** -125 * 0.75, 2.0 ** 126, 2.0 ** 126 * 1.5)
+    for c1 in (1.0, 0.0371, 3.0517578e-5, 7.5e3, float(rng.uniform(0.01, 0.2))) + edges:
         c1 = np.float32(c1)
         q = (vals.astype(np.float64) * np.float64(c1)).astype(np.float32)   # w near c1 * point
         pad = (-q.size) % 63
