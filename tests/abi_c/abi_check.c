@@ -2,9 +2,12 @@
  * A plain C99 client of libqlora: include/qlora.h must compile as C, every
  * entry point must link, and the host-only calls must behave as the header
  * documents. Nothing here launches a kernel, so it runs without a GPU.
- * Exit status 0 and "ok" on stdout when every check holds; otherwise the
- * first failing check is printed and the status is 1.
+ * It also prints the size and field offsets of each struct of the header, one
+ * "layout" line per struct, for a binding to compare its own mirrors with.
+ * Exit status 0 and "ok" as the last line when every check holds; otherwise
+ * each failing check is printed and the status is 1.
  */
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -106,6 +109,23 @@ int main(void) {
     }
     CHECK(strcmp(qlora_status_string((qlora_status_t)12345), "QLORA_ERR_UNKNOWN") == 0);
   }
+
+  /* the layouts a binding must mirror: "layout <struct> <size> <field>=<offset> ..." */
+  printf("layout qlora_nf4_t %u rows=%u cols=%u codes=%u scale8=%u scale2=%u\n", (unsigned)sizeof(qlora_nf4_t),
+         (unsigned)offsetof(qlora_nf4_t, rows), (unsigned)offsetof(qlora_nf4_t, cols),
+         (unsigned)offsetof(qlora_nf4_t, codes), (unsigned)offsetof(qlora_nf4_t, scale8),
+         (unsigned)offsetof(qlora_nf4_t, scale2));
+  printf("layout qlora_linear_problem_t %u W=%u X=%u A=%u B=%u r=%u s=%u Y=%u sU_out=%u\n",
+         (unsigned)sizeof(qlora_linear_problem_t), (unsigned)offsetof(qlora_linear_problem_t, W),
+         (unsigned)offsetof(qlora_linear_problem_t, X), (unsigned)offsetof(qlora_linear_problem_t, A),
+         (unsigned)offsetof(qlora_linear_problem_t, B), (unsigned)offsetof(qlora_linear_problem_t, r),
+         (unsigned)offsetof(qlora_linear_problem_t, s), (unsigned)offsetof(qlora_linear_problem_t, Y),
+         (unsigned)offsetof(qlora_linear_problem_t, sU_out));
+  printf("layout qlora_adamw8_tensor_t %u p=%u p_bf16=%u m_q=%u v_q=%u m_scale=%u v_scale=%u\n",
+         (unsigned)sizeof(qlora_adamw8_tensor_t), (unsigned)offsetof(qlora_adamw8_tensor_t, p),
+         (unsigned)offsetof(qlora_adamw8_tensor_t, p_bf16), (unsigned)offsetof(qlora_adamw8_tensor_t, m_q),
+         (unsigned)offsetof(qlora_adamw8_tensor_t, v_q), (unsigned)offsetof(qlora_adamw8_tensor_t, m_scale),
+         (unsigned)offsetof(qlora_adamw8_tensor_t, v_scale));
 
   if (failures) return 1;
   printf("ok\n");
